@@ -1,0 +1,193 @@
+"""CPU oracle for load-balanced MoE token dispatch/combine -- TEST INFRASTRUCTURE.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's CPU
+baseline leg may import this package.  The product path (the CUDA library and
+its Python binding) never imports, calls or falls back to it.
+
+The arithmetic lives in ``zb_oracle.c`` (plain C, single-threaded, compiled
+with ``-ffp-contract=off`` and without fast-math); this module only compiles it
+with gcc, marshals numpy arrays and returns the results.  Every function of
+the C file cites the web-page passage it follows (Zepp 4.1 eq. (1); ISER-MoE
+HALO-Q Scheduler; MoonEP "What MoonEP enforces and how").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "zb_oracle.c")
+_LIB = os.path.join(_HERE, "libzb_oracle.so")
+
+OK = 0
+UNBALANCED = 1
+ERR_INVALID = -1
+ERR_CAPACITY = -2
+ERR_BAD_ID = -3
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (no CUDA involved) and return the .so path."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-Wall", "-ffp-contract=off", "-fno-fast-math",
+             "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [("P", ctypes.c_int), ("E", ctypes.c_int), ("K", ctypes.c_int),
+                ("S", ctypes.c_int), ("H", ctypes.c_int), ("R", ctypes.c_int),
+                ("C", ctypes.c_double), ("gpus_per_node", ctypes.c_int),
+                ("cap_rows", ctypes.c_int)]
+
+
+_P32 = ctypes.POINTER(ctypes.c_int32)
+
+
+class _Out(ctypes.Structure):
+    _fields_ = [("cnt", _P32), ("rep_expert", _P32), ("rep_quota", _P32),
+                ("home_quota", _P32), ("load_before", _P32), ("load_after", _P32),
+                ("cu_seqlens", _P32), ("dst_row", _P32), ("row_src", _P32), ("M", _P32),
+                ("locality_cost", ctypes.c_int64), ("max_load", ctypes.c_int32),
+                ("n_replicas", ctypes.c_int32), ("n_iters", ctypes.c_int32),
+                ("water_level", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        lib.zbo_validate.argtypes = [ctypes.POINTER(_Cfg)]
+        lib.zbo_plan.argtypes = [ctypes.POINTER(_Cfg), _P32, ctypes.POINTER(_Out)]
+        vp = ctypes.c_void_p
+        lib.zbo_dispatch.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp]
+        lib.zbo_dispatch.restype = None
+        lib.zbo_combine.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, vp]
+        lib.zbo_combine.restype = None
+        lib.zbo_f32_to_bf16.argtypes = [ctypes.c_float]
+        lib.zbo_f32_to_bf16.restype = ctypes.c_uint16
+        lib.zbo_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        lib.zbo_bf16_to_f32.restype = ctypes.c_float
+        d = ctypes.POINTER(ctypes.c_double)
+        lib.zbo_metrics.argtypes = [ctypes.POINTER(_Cfg), _P32, _P32, _P32, d, d, d, d]
+        lib.zbo_metrics.restype = None
+        _lib = lib
+    return _lib
+
+
+@dataclass
+class Config:
+    """Problem shape.  ``cap_rows`` defaults to S*K (the water level)."""
+    P: int
+    E: int
+    K: int
+    S: int
+    H: int
+    R: int
+    C: float = 0.0
+    gpus_per_node: int = 1
+    cap_rows: int | None = None
+
+    def cap(self) -> int:
+        return self.S * self.K if self.cap_rows is None else self.cap_rows
+
+    def c(self) -> _Cfg:
+        return _Cfg(self.P, self.E, self.K, self.S, self.H, self.R, float(self.C),
+                    self.gpus_per_node, self.cap())
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags.c_contiguous
+    return a.ctypes.data_as(_P32)
+
+
+def validate(cfg: Config) -> int:
+    return int(_load().zbo_validate(ctypes.byref(cfg.c())))
+
+
+def plan(cfg: Config, ids: np.ndarray, want_M: bool = True) -> dict:
+    """Steps 1-3 on host arrays.  ``ids`` is int32 ``[P,S,K]``.
+
+    Returns a dict with ``status`` and the plan tables (numpy int32 arrays
+    shaped as the C comments state), ``M`` ``[E,P,P]`` when requested, and the
+    scalars ``locality_cost``, ``max_load``, ``n_replicas``, ``n_iters``, ``T``.
+    """
+    lib = _load()
+    P, E, K, S, R = cfg.P, cfg.E, cfg.K, cfg.S, cfg.R
+    Eh = E // max(P, 1)
+    cap = cfg.cap()
+    ids = np.ascontiguousarray(ids, dtype=np.int32).reshape(P, S, K)
+    r = dict(
+        cnt=np.zeros((P, E), np.int32), rep_expert=np.zeros((P, R), np.int32),
+        rep_quota=np.zeros((P, R), np.int32), home_quota=np.zeros(E, np.int32),
+        load_before=np.zeros(P, np.int32), load_after=np.zeros(P, np.int32),
+        cu_seqlens=np.zeros((P, Eh + R + 1), np.int32), dst_row=np.zeros((P, S, K), np.int32),
+        row_src=np.zeros((P, cap), np.int32))
+    if want_M:
+        r["M"] = np.zeros((E, P, P), np.int32)
+    out = _Out(*[_ptr(r[k]) for k in ("cnt", "rep_expert", "rep_quota", "home_quota",
+                                       "load_before", "load_after", "cu_seqlens",
+                                       "dst_row", "row_src")],
+               _ptr(r["M"]) if want_M else _P32(), 0, 0, 0, 0, 0)
+    st = lib.zbo_plan(ctypes.byref(cfg.c()), _ptr(ids), ctypes.byref(out))
+    r.update(status=int(st), locality_cost=int(out.locality_cost), max_load=int(out.max_load),
+             n_replicas=int(out.n_replicas), n_iters=int(out.n_iters), T=int(out.water_level))
+    return r
+
+
+def dispatch(cfg: Config, dst_row: np.ndarray, hidden_bits: np.ndarray,
+             buf_bits: np.ndarray | None = None) -> np.ndarray:
+    """Step 4.  ``hidden_bits`` is uint16 (bf16 bit patterns) ``[P,S,H]``.
+
+    Writes into ``buf_bits`` (uint16 ``[P,cap,H]``) if given, else into a
+    zero-filled new buffer, and returns it.
+    """
+    P, S, H = cfg.P, cfg.S, cfg.H
+    hidden_bits = np.ascontiguousarray(hidden_bits, dtype=np.uint16).reshape(P, S, H)
+    dst_row = np.ascontiguousarray(dst_row, dtype=np.int32)
+    if buf_bits is None:
+        buf_bits = np.zeros((P, cfg.cap(), H), np.uint16)
+    assert buf_bits.dtype == np.uint16 and buf_bits.flags.c_contiguous
+    _load().zbo_dispatch(ctypes.byref(cfg.c()), dst_row.ctypes.data, hidden_bits.ctypes.data,
+                         buf_bits.ctypes.data)
+    return buf_bits
+
+
+def combine(cfg: Config, dst_row: np.ndarray, y_bits: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """Step 5.  ``y_bits`` uint16 ``[rows,H]`` indexed by ``dst_row``; ``w``
+    float32 ``[P,S,K]``.  Returns uint16 ``[P,S,H]``."""
+    P, S, H = cfg.P, cfg.S, cfg.H
+    dst_row = np.ascontiguousarray(dst_row, dtype=np.int32)
+    y_bits = np.ascontiguousarray(y_bits, dtype=np.uint16)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    out = np.zeros((P, S, H), np.uint16)
+    _load().zbo_combine(ctypes.byref(cfg.c()), dst_row.ctypes.data, y_bits.ctypes.data,
+                        w.ctypes.data, out.ctypes.data)
+    return out
+
+
+def f32_to_bf16(x: float) -> int:
+    return int(_load().zbo_f32_to_bf16(ctypes.c_float(x)))
+
+
+def bf16_to_f32(b: int) -> float:
+    return float(_load().zbo_bf16_to_f32(ctypes.c_uint16(b)))
+
+
+def metrics(cfg: Config, p: dict) -> dict:
+    lib = _load()
+    vals = [ctypes.c_double() for _ in range(4)]
+    lib.zbo_metrics(ctypes.byref(cfg.c()), _ptr(p["cnt"]), _ptr(p["load_before"]),
+                    _ptr(p["load_after"]), *[ctypes.byref(v) for v in vals])
+    return dict(r_imb_before=vals[0].value, r_imb_after=vals[1].value, maxvio=vals[2].value,
+                excess_removed=vals[3].value)

@@ -1,0 +1,493 @@
+/*
+ * zb_oracle.c -- the CPU oracle for load-balanced MoE token dispatch/combine.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the plain, slow, single-threaded
+ * statement of what the device path computes.  Only the test suite, the smoke
+ * check and the benchmark's CPU-baseline leg may load it.  The product path
+ * never calls it, links it or falls back to it, and it shares no code, header
+ * or table with the CUDA library: it does not include the library's header and
+ * defines its own structs.
+ *
+ * Sources (web pages; each function cites the passage it follows):
+ *  [ZEPP]  Zepp summary page, "Methodology / 4.1 Expert Placement and Token
+ *          Routing" (R replica slots per GPU, hierarchical round-robin
+ *          placement, locality-preferred routing eq. (1)).
+ *  [ISER]  "ISER-MoE: Dynamic In-Switch Replication of Hot Experts for Load
+ *          Balancing in Expert-Parallel", "Methodology / HALO-Q Scheduler"
+ *          (Objective 1 water level T, stage 1 count exchange, stage 2 greedy
+ *          placement of the busiest rank's heaviest home expert, stage 3 slot
+ *          colouring by the smallest free index, stage 5 local-first route
+ *          rewrite), "Background" (rank imbalance R = max/mean).
+ *  [MOON]  "MoonEP: Planner-Enforced SxK Token Balance and Zero-Copy Buffers
+ *          to Fix MoE Skew", "What MoonEP enforces and how" (every rank gets
+ *          exactly S*K rows; the planner emits cu_seqlens; fixed-shape
+ *          expert-grouped buffers), "Variables and core terms" (maxvio).
+ *
+ * Readings taken where the pages leave a step open (each also listed in the
+ * design notes of the repository):
+ *  - home(e) = floor(e / (E/P)): experts are partitioned contiguously.
+ *  - "heaviest home expert" = the largest remaining home quota, ties to the
+ *    lowest expert id; the receiver is the eligible rank with the most room
+ *    (lowest load), ties to the lowest rank; with nodes, a rank on a node that
+ *    does not yet hold the expert comes first (round-robin across nodes).
+ *  - quotas are delivered exactly (|sum_i M_ij - q_j| = 0 <= C*q_j), because
+ *    T = S*K leaves no slack in the fixed S*K buffers.
+ *  - rows inside a group are ordered by (source rank, flat index s*K+k).
+ *  - combine: acc = +0.0f; acc = fmaf(w_k, y_k, acc) for k = 0..K-1; the
+ *    result is rounded to bf16 to nearest, ties to even.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fPIC -shared zb_oracle.c -lm
+ * (no -ffast-math: the combine must use one correctly rounded fmaf per term).
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <math.h>
+
+#define ZBO_OK 0
+#define ZBO_UNBALANCED 1
+#define ZBO_ERR_INVALID (-1)
+#define ZBO_ERR_CAPACITY (-2)
+#define ZBO_ERR_BAD_ID (-3)
+#define ZBO_ERR_INTERNAL (-9)
+
+typedef struct {
+  int P;             /* expert-parallel ranks (virtual on one GPU) */
+  int E;             /* experts; E/P home experts per rank */
+  int K;             /* top-K routed experts per token */
+  int S;             /* tokens per rank */
+  int H;             /* hidden width (bf16 elements per row) */
+  int R;             /* replica (helper) slots per rank */
+  double C;          /* relaxation ratio of eq. (1); validated, recorded */
+  int gpus_per_node; /* 1 = flat locality cost; >1 = two-level cost */
+  int cap_rows;      /* rows of each rank's receive buffer (>= S*K) */
+} zbo_config;
+
+typedef struct {
+  int32_t *cnt;         /* [P][E]     routed entries of rank i to expert e */
+  int32_t *rep_expert;  /* [P][R]     expert held in helper slot, -1 = empty */
+  int32_t *rep_quota;   /* [P][R]     rows the helper slot receives */
+  int32_t *home_quota;  /* [E]        rows the home copy receives */
+  int32_t *load_before; /* [P]        L_j before planning */
+  int32_t *load_after;  /* [P]        rank load after planning */
+  int32_t *cu_seqlens;  /* [P][E/P+R+1] exclusive prefix of group sizes */
+  int32_t *dst_row;     /* [P][S][K]  j*cap + row, -1 when not assigned */
+  int32_t *row_src;     /* [P][cap]   g=(i*S+s)*K+k or -1 (may be NULL) */
+  int32_t *M;           /* [E][P][P]  transport M^e_ij (may be NULL) */
+  int64_t locality_cost;
+  int32_t max_load;
+  int32_t n_replicas;
+  int32_t n_iters;
+  int32_t water_level;
+} zbo_plan_out;
+
+/* ---------------------------------------------------------------- helpers */
+
+static int home_of(const zbo_config *c, int e) { return e / (c->E / c->P); }
+static int node_of(const zbo_config *c, int r) { return r / c->gpus_per_node; }
+
+/* a_ij of eq. (1) [ZEPP 4.1]: a is inverse bandwidth.  0 on the same GPU;
+ * with one GPU per node every other rank costs 1; with several GPUs per node
+ * a rank on the same node costs 1 and a rank on another node costs 4. */
+static int cost_a(const zbo_config *c, int i, int j) {
+  if (i == j) return 0;
+  if (c->gpus_per_node > 1 && node_of(c, i) != node_of(c, j)) return 4;
+  return 1;
+}
+
+int zbo_validate(const zbo_config *c) {
+  if (c->P < 1 || c->P > 32) return ZBO_ERR_INVALID;
+  if (c->E < c->P || c->E > 384 || c->E % c->P != 0) return ZBO_ERR_INVALID;
+  if (c->K < 1 || c->K > 16) return ZBO_ERR_INVALID;
+  if (c->S < 0) return ZBO_ERR_INVALID;
+  if (c->H < 8 || c->H % 8 != 0) return ZBO_ERR_INVALID;
+  if (c->R < 0 || c->R > c->P - 1) return ZBO_ERR_INVALID;
+  if (!(c->C >= 0.0 && c->C < 1.0)) return ZBO_ERR_INVALID;
+  if (c->gpus_per_node < 1 || c->P % c->gpus_per_node != 0) return ZBO_ERR_INVALID;
+  if ((int64_t)c->S * c->K > INT32_MAX) return ZBO_ERR_INVALID;
+  if (c->cap_rows < c->S * c->K) return ZBO_ERR_INVALID;
+  if ((int64_t)c->P * c->S * c->K > INT32_MAX) return ZBO_ERR_INVALID;
+  if ((int64_t)c->P * c->cap_rows > INT32_MAX) return ZBO_ERR_INVALID;
+  return ZBO_OK;
+}
+
+/* -------------------------------------------------- step 1: the histogram */
+
+/* cnt[i][e] = #{(s,k) : ids[i,s,k] = e}: the per-rank route counts that
+ * HALO-Q stage 1 exchanges [ISER, HALO-Q Scheduler, stage 1]. */
+static int histogram(const zbo_config *c, const int32_t *ids, int32_t *cnt) {
+  memset(cnt, 0, sizeof(int32_t) * (size_t)c->P * c->E);
+  for (int i = 0; i < c->P; i++)
+    for (int64_t f = 0; f < (int64_t)c->S * c->K; f++) {
+      int32_t e = ids[(int64_t)i * c->S * c->K + f];
+      if (e < 0 || e >= c->E) return ZBO_ERR_BAD_ID;
+      cnt[(size_t)i * c->E + e] += 1;
+    }
+  return ZBO_OK;
+}
+
+/* ------------------------------------------ step 2: the greedy planner */
+
+typedef struct {
+  const zbo_config *c;
+  int32_t *rep_expert, *rep_quota; /* [P][R] */
+  int *nfill;                      /* filled slots per rank */
+} slots_t;
+
+static int holds_replica(const slots_t *st, int r, int e) {
+  for (int s = 0; s < st->nfill[r]; s++)
+    if (st->rep_expert[r * st->c->R + s] == e) return 1;
+  return 0;
+}
+
+/* Does the node of rank r already hold expert e, as home or as replica?
+ * Placing where this is false first spreads replicas round-robin across
+ * nodes before GPUs within a node [ZEPP 4.1, hierarchical placement]. */
+static int node_covers(const slots_t *st, int r, int e) {
+  const zbo_config *c = st->c;
+  int n = node_of(c, r);
+  if (node_of(c, home_of(c, e)) == n) return 1;
+  for (int q = n * c->gpus_per_node; q < (n + 1) * c->gpus_per_node; q++)
+    if (holds_replica(st, q, e)) return 1;
+  return 0;
+}
+
+/* Greedy replica placement [ISER, HALO-Q Scheduler, Objective 1 and stage 2;
+ * ZEPP 4.1 "R extra slots per GPU"; slot colouring by the smallest free index,
+ * ISER stage 3].  Repeatedly: the busiest rank d (ties: lowest rank) offers
+ * its heaviest home expert (largest remaining home quota, ties: lowest id)
+ * that some rank can take; the receiver is the eligible rank with the most
+ * room (node coverage first when there are nodes), and receives
+ * m = min(load[d]-T, T-load[r], hq[e]) of that expert's rows in its lowest
+ * free slot.  A donor for which no expert has an eligible receiver is marked
+ * stuck.  Stops when the busiest non-stuck rank is at or below T. */
+static void greedy_place(const zbo_config *c, int32_t T, int32_t *load, int32_t *hq,
+                         int32_t *rep_expert, int32_t *rep_quota, int32_t *n_iters) {
+  const int P = c->P, E = c->E, R = c->R, Eh = E / P;
+  int *nfill = calloc((size_t)P, sizeof(int));
+  int *stuck = calloc((size_t)P, sizeof(int));
+  int *order = malloc(sizeof(int) * (size_t)Eh);
+  slots_t st = {c, rep_expert, rep_quota, nfill};
+  for (int x = 0; x < P * R; x++) { rep_expert[x] = -1; rep_quota[x] = 0; }
+  *n_iters = 0;
+  for (;;) {
+    int d = -1;
+    for (int j = 0; j < P; j++)
+      if (!stuck[j] && (d < 0 || load[j] > load[d])) d = j;
+    if (d < 0 || load[d] <= T) break;
+    *n_iters += 1;
+
+    /* d's home experts with quota left, heaviest first (insertion sort). */
+    int n = 0;
+    for (int e = d * Eh; e < (d + 1) * Eh; e++) {
+      if (hq[e] <= 0) continue;
+      int p = n++;
+      while (p > 0 && (hq[order[p - 1]] < hq[e])) { order[p] = order[p - 1]; p--; }
+      order[p] = e;
+    }
+
+    int pick_e = -1, pick_r = -1;
+    for (int t = 0; t < n && pick_e < 0; t++) {
+      int e = order[t];
+      int best = -1, best_cov = 0;
+      for (int r = 0; r < P; r++) {
+        if (r == d || nfill[r] >= R || load[r] >= T || holds_replica(&st, r, e)) continue;
+        int cov = node_covers(&st, r, e);
+        if (best < 0 || cov < best_cov || (cov == best_cov && load[r] < load[best])) {
+          best = r;
+          best_cov = cov;
+        }
+      }
+      if (best >= 0) { pick_e = e; pick_r = best; }
+    }
+    if (pick_e < 0) { stuck[d] = 1; continue; }
+
+    int32_t m = load[d] - T;
+    if (T - load[pick_r] < m) m = T - load[pick_r];
+    if (hq[pick_e] < m) m = hq[pick_e];
+    int slot = nfill[pick_r]++;
+    rep_expert[pick_r * R + slot] = pick_e;
+    rep_quota[pick_r * R + slot] = m;
+    load[pick_r] += m;
+    load[d] -= m;
+    hq[pick_e] -= m;
+  }
+  free(order);
+  free(stuck);
+  free(nfill);
+}
+
+/* ------------------------- step 3: transport, groups, cu_seqlens, rows */
+
+typedef struct { int rank, group; int32_t quota; } host_t;
+
+/* The hosts of expert e in ascending rank order: its home rank (group
+ * e - home*Eh) and every rank holding a replica (group Eh + slot). */
+static int hosts_of(const zbo_config *c, int e, const int32_t *home_quota,
+                    const int32_t *rep_expert, const int32_t *rep_quota, host_t *out) {
+  const int Eh = c->E / c->P;
+  int n = 0, h = home_of(c, e);
+  for (int j = 0; j < c->P; j++) {
+    if (j == h) {
+      out[n].rank = j; out[n].group = e - h * Eh; out[n].quota = home_quota[e]; n++;
+    }
+    for (int s = 0; s < c->R; s++)
+      if (rep_expert[j * c->R + s] == e) {
+        out[n].rank = j; out[n].group = Eh + s; out[n].quota = rep_quota[j * c->R + s]; n++;
+      }
+  }
+  return n;
+}
+
+/* Locality-preferred routing, eq. (1) [ZEPP 4.1] with the local-first route
+ * rewrite [ISER, HALO-Q stage 5]: serve each host's quota from the host's own
+ * rank first (a=0), then for every cost level in increasing order, hosts in
+ * ascending rank, sources in ascending rank.  Writes M[i*P+j] for expert e. */
+static int transport(const zbo_config *c, const int32_t *cnt, int e,
+                     const host_t *hosts, int nh, int32_t *M) {
+  const int P = c->P;
+  int32_t dres[32], qres[33];
+  memset(M, 0, sizeof(int32_t) * (size_t)P * P);
+  for (int i = 0; i < P; i++) dres[i] = cnt[(size_t)i * c->E + e];
+  for (int h = 0; h < nh; h++) qres[h] = hosts[h].quota;
+  for (int h = 0; h < nh; h++) {
+    int j = hosts[h].rank;
+    int32_t take = dres[j] < qres[h] ? dres[j] : qres[h];
+    M[j * P + j] += take; dres[j] -= take; qres[h] -= take;
+  }
+  int levels[2] = {1, 4};
+  int nlev = c->gpus_per_node > 1 ? 2 : 1;
+  for (int l = 0; l < nlev; l++)
+    for (int h = 0; h < nh; h++) {
+      int j = hosts[h].rank;
+      for (int i = 0; i < P; i++) {
+        if (cost_a(c, i, j) != levels[l]) continue;
+        int32_t take = dres[i] < qres[h] ? dres[i] : qres[h];
+        M[i * P + j] += take; dres[i] -= take; qres[h] -= take;
+      }
+    }
+  for (int i = 0; i < P; i++) if (dres[i] != 0) return ZBO_ERR_INTERNAL;
+  for (int h = 0; h < nh; h++) if (qres[h] != 0) return ZBO_ERR_INTERNAL;
+  return ZBO_OK;
+}
+
+/* The whole plan: steps 1-3.  Returns ZBO_OK, ZBO_UNBALANCED (some rank stays
+ * above T because R slots do not permit T), or an error.  On
+ * ZBO_ERR_CAPACITY the plan tables are valid but dst_row/row_src are all -1. */
+int zbo_plan(const zbo_config *c, const int32_t *ids, zbo_plan_out *out) {
+  int rc = zbo_validate(c);
+  if (rc) return rc;
+  const int P = c->P, E = c->E, R = c->R, Eh = E / P, G = Eh + R;
+  const int64_t NK = (int64_t)c->S * c->K;
+
+  rc = histogram(c, ids, out->cnt);
+  if (rc) return rc;
+
+  /* T_e = sum_i cnt[i][e];  L_j = sum over j's home experts of T_e. */
+  int32_t *Te = calloc((size_t)E, sizeof(int32_t));
+  for (int i = 0; i < P; i++)
+    for (int e = 0; e < E; e++) Te[e] += out->cnt[(size_t)i * E + e];
+  int64_t sumL = 0;
+  for (int j = 0; j < P; j++) {
+    int32_t L = 0;
+    for (int e = j * Eh; e < (j + 1) * Eh; e++) L += Te[e];
+    out->load_before[j] = L;
+    out->load_after[j] = L;
+    sumL += L;
+  }
+  /* Water level T = ceil(sum_r L_r / P) [ISER, HALO-Q Objective 1]. */
+  int32_t T = (int32_t)((sumL + P - 1) / P);
+  out->water_level = T;
+
+  for (int e = 0; e < E; e++) out->home_quota[e] = Te[e];
+  greedy_place(c, T, out->load_after, out->home_quota, out->rep_expert, out->rep_quota,
+               &out->n_iters);
+
+  out->max_load = 0;
+  out->n_replicas = 0;
+  for (int j = 0; j < P; j++)
+    if (out->load_after[j] > out->max_load) out->max_load = out->load_after[j];
+  for (int x = 0; x < P * R; x++) out->n_replicas += out->rep_expert[x] >= 0;
+
+  /* Transport per expert, kept whole: Mall[e][i][j]. */
+  int32_t *Mall = calloc((size_t)E * P * P, sizeof(int32_t));
+  host_t hosts[33];
+  out->locality_cost = 0;
+  for (int e = 0; e < E; e++) {
+    int nh = hosts_of(c, e, out->home_quota, out->rep_expert, out->rep_quota, hosts);
+    rc = transport(c, out->cnt, e, hosts, nh, Mall + (size_t)e * P * P);
+    if (rc) { free(Mall); free(Te); return rc; }
+    for (int i = 0; i < P; i++)
+      for (int j = 0; j < P; j++)
+        out->locality_cost += (int64_t)cost_a(c, i, j) * Mall[((size_t)e * P + i) * P + j];
+  }
+  if (out->M) memcpy(out->M, Mall, sizeof(int32_t) * (size_t)E * P * P);
+
+  /* Groups of rank j: home experts j*Eh .. j*Eh+Eh-1, then slots 0..R-1.
+   * cu_seqlens[j] is the exclusive prefix of the rows each group receives,
+   * sum_i M^e_ij [MOON, "the planner returns cu_seqlens"]. */
+  for (int j = 0; j < P; j++) {
+    int32_t *cu = out->cu_seqlens + (size_t)j * (G + 1);
+    cu[0] = 0;
+    for (int g = 0; g < G; g++) {
+      int e = g < Eh ? j * Eh + g : out->rep_expert[j * R + (g - Eh)];
+      int32_t recv = 0;
+      if (e >= 0)
+        for (int i = 0; i < P; i++) recv += Mall[((size_t)e * P + i) * P + j];
+      cu[g + 1] = cu[g] + recv;
+    }
+  }
+
+  int status = out->max_load > T ? ZBO_UNBALANCED : ZBO_OK;
+  const int64_t cap = c->cap_rows;
+  if (out->row_src)
+    for (int64_t x = 0; x < (int64_t)P * cap; x++) out->row_src[x] = -1;
+  if (out->max_load > c->cap_rows) {
+    for (int64_t x = 0; x < (int64_t)P * NK; x++) out->dst_row[x] = -1;
+    free(Mall); free(Te);
+    return ZBO_ERR_CAPACITY;
+  }
+
+  /* Rows.  Source i walks its entries of expert e in flat order f = s*K+k
+   * and fills its hosts in order of (a_ij, j): the first M_{i,h1} entries go
+   * to h1, the next M_{i,h2} to h2, ...  Inside host j's group, source i's
+   * segment starts after the rows of sources i' < i. */
+  int32_t *cursor = calloc((size_t)E, sizeof(int32_t)); /* index into order */
+  int32_t *taken = calloc((size_t)E, sizeof(int32_t));  /* used in current host */
+  host_t *hl = malloc(sizeof(host_t) * (size_t)E * 33);
+  int *nhl = calloc((size_t)E, sizeof(int));
+  for (int e = 0; e < E; e++)
+    nhl[e] = hosts_of(c, e, out->home_quota, out->rep_expert, out->rep_quota, hl + (size_t)e * 33);
+  for (int i = 0; i < P; i++) {
+    /* host order of source i for each expert: a ascending, then rank */
+    int32_t *ord = malloc(sizeof(int32_t) * (size_t)E * 33);
+    for (int e = 0; e < E; e++) {
+      int n = 0;
+      for (int a = 0; a <= 4; a++)
+        for (int h = 0; h < nhl[e]; h++)
+          if (cost_a(c, i, hl[(size_t)e * 33 + h].rank) == a) ord[(size_t)e * 33 + n++] = h;
+      cursor[e] = 0;
+      taken[e] = 0;
+    }
+    for (int64_t f = 0; f < NK; f++) {
+      int64_t gidx = (int64_t)i * NK + f;
+      int e = ids[gidx];
+      int h, j;
+      int32_t Mij;
+      for (;;) {
+        h = ord[(size_t)e * 33 + cursor[e]];
+        j = hl[(size_t)e * 33 + h].rank;
+        Mij = Mall[((size_t)e * P + i) * P + j];
+        if (taken[e] < Mij) break;
+        cursor[e] += 1;
+        taken[e] = 0;
+      }
+      int32_t seg = 0;
+      for (int ip = 0; ip < i; ip++) seg += Mall[((size_t)e * P + ip) * P + j];
+      int32_t row = out->cu_seqlens[(size_t)j * (G + 1) + hl[(size_t)e * 33 + h].group] + seg +
+                    taken[e];
+      taken[e] += 1;
+      int32_t dst = (int32_t)(j * cap + row);
+      out->dst_row[gidx] = dst;
+      if (out->row_src) out->row_src[dst] = (int32_t)gidx;
+    }
+    free(ord);
+  }
+  free(nhl); free(hl); free(taken); free(cursor);
+  free(Mall); free(Te);
+  return status;
+}
+
+/* ------------------------------------------------ bf16 (IEEE definition) */
+
+/* bf16 is the upper half of an IEEE binary32: widening is exact. */
+float zbo_bf16_to_f32(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+/* binary32 -> bf16, round to nearest, ties to even.  Keep the upper 16 bits;
+ * the lower 16 bits are the discarded fraction r.  Round up when r is more
+ * than half an ulp, or exactly half and the kept last bit is odd.  Rounding up
+ * is an integer increment of the kept bits, which carries into the exponent
+ * (and from the largest finite value to infinity) as IEEE prescribes.  NaN
+ * stays NaN (returned as the canonical quiet NaN 0x7FC0 with its sign). */
+uint16_t zbo_f32_to_bf16(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu) != 0)
+    return (uint16_t)(((u >> 16) & 0x8000u) | 0x7FC0u);
+  uint32_t kept = u >> 16;
+  uint32_t r = u & 0xFFFFu;
+  if (r > 0x8000u || (r == 0x8000u && (kept & 1u))) kept += 1;
+  return (uint16_t)kept;
+}
+
+/* ------------------------------------------------- step 4: the dispatch */
+
+/* buf[dst_row[i,s,k]] = hidden[i,s], bit for bit: the zero-copy write of a
+ * token row into the fixed-shape, expert-grouped buffer of its destination
+ * rank [MOON, "What MoonEP enforces and how"].  Rows nobody is routed to are
+ * not touched. */
+void zbo_dispatch(const zbo_config *c, const int32_t *dst_row, const uint16_t *hidden,
+                  uint16_t *buf) {
+  const int64_t H = c->H;
+  for (int64_t t = 0; t < (int64_t)c->P * c->S; t++)
+    for (int k = 0; k < c->K; k++) {
+      int32_t row = dst_row[t * c->K + k];
+      if (row < 0) continue;
+      memcpy(buf + (int64_t)row * H, hidden + t * H, sizeof(uint16_t) * (size_t)H);
+    }
+}
+
+/* ------------------------------------------------- step 5: the combine */
+
+/* out[t] = bf16( fmaf(w_{K-1}, y_{K-1}, ... fmaf(w_0, y_0, +0.0f)) ): the
+ * inverse of dispatch, a gate-weighted sum of the token's K expert rows in the
+ * fixed order k = 0..K-1, one rounding per fused multiply-add, accumulated in
+ * binary32 and rounded once to bf16 [ZEPP 4.2 merge/combine; MOON mechanics]. */
+void zbo_combine(const zbo_config *c, const int32_t *dst_row, const uint16_t *y,
+                 const float *w, uint16_t *out) {
+  const int64_t H = c->H;
+  for (int64_t t = 0; t < (int64_t)c->P * c->S; t++)
+    for (int64_t h = 0; h < H; h++) {
+      float acc = 0.0f;
+      for (int k = 0; k < c->K; k++) {
+        int64_t row = dst_row[t * c->K + k];
+        acc = fmaf(w[t * c->K + k], zbo_bf16_to_f32(y[row * H + h]), acc);
+      }
+      out[t * H + h] = zbo_f32_to_bf16(acc);
+    }
+}
+
+/* ------------------------------------------------------------- metrics */
+
+/* R_imb = max_j L_j / mean_j L_j [ISER, Background]; maxvio =
+ * max_e T_e / mean_e T_e - 1 [MOON, Variables and core terms]; excess removed
+ * = (max_before - max_after) / (max_before - T) [ISER, Table E1]. */
+void zbo_metrics(const zbo_config *c, const int32_t *cnt, const int32_t *load_before,
+                 const int32_t *load_after, double *r_before, double *r_after, double *maxvio,
+                 double *excess_removed) {
+  double sum = 0, mb = 0, ma = 0;
+  for (int j = 0; j < c->P; j++) {
+    sum += load_before[j];
+    if (load_before[j] > mb) mb = load_before[j];
+    if (load_after[j] > ma) ma = load_after[j];
+  }
+  double mean = sum / c->P;
+  *r_before = mean > 0 ? mb / mean : 1.0;
+  *r_after = mean > 0 ? ma / mean : 1.0;
+  double tmax = 0, tsum = 0;
+  for (int e = 0; e < c->E; e++) {
+    double te = 0;
+    for (int i = 0; i < c->P; i++) te += cnt[(size_t)i * c->E + e];
+    tsum += te;
+    if (te > tmax) tmax = te;
+  }
+  double tbar = tsum / c->E;
+  *maxvio = tbar > 0 ? tmax / tbar - 1.0 : 0.0;
+  double T = ceil(sum / c->P);
+  *excess_removed = mb > T ? (mb - ma) / (mb - T) : 1.0;
+}
