@@ -1,0 +1,403 @@
+"""Benchmark: plan + dispatch + combine tokens/s on B200, with the HBM roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one invocation of the whole hot path (histogram, greedy replica
+plan, assignment, dispatch scatter, combine gather) on the mid workload: P=8
+virtual ranks, E=64, K=6, S=4096 tokens per rank, H=2048 bf16, R=2, C=0.1,
+Zipf s=1.2 popularity with a per-seed permuted ranking.  The expert outputs fed
+to the combine are the dispatched rows themselves (identity experts), so the
+step moves exactly the dispatch and combine traffic.
+
+* ``value``: tokens/s over all ranks, device-timed with CUDA events with the
+  inputs resident in HBM; L2 (126 MB) is flushed by a 256 MB write before
+  every step, outside the timed events.
+* ``e2e``: the same metric through the public API with pinned host buffers:
+  each step copies ids, weights and hidden rows host->device, runs the path,
+  and copies the combined rows and the plan status back.
+* ``roofline``: the dominant kernel's algorithmic bytes per launch over its
+  event-timed duration, against the measured HBM copy bandwidth.
+* ``cpu_baseline``: the CPU oracle (single thread) on full steps of the same
+  workload, rank 0 at N=1 only.
+
+With ``--impl reference`` the CPU oracle itself is timed on the same workload
+(rank 0 only; other ranks exit).  With N>1 (torchrun), every rank runs an
+independent replica on its own GPU (the path has no cross-rank exchange on one
+GPU); ``value`` is the sum of tokens over ranks divided by the slowest rank's
+time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "plan+dispatch+combine tokens/s at 1 GPU; achieved HBM GB/s vs B200 peak"
+UNIT = "tokens/s"
+WORKLOAD = "mid"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def workload_desc(wl) -> str:
+    return (f"{wl.name}: P={wl.P} E={wl.E} K={wl.K} S={wl.S} H={wl.H} R={wl.R} C={wl.C}, "
+            f"Zipf s={wl.zipf_s} popularity, permuted ranking, seed 0")
+
+
+def algorithmic_bytes(wl) -> dict:
+    """Bytes each step must move at least (bf16 rows, int32 indices, fp32 gates)."""
+    P, S, K, H = wl.P, wl.S, wl.K, wl.H
+    N = P * S * K
+    tok_rows = P * S * H * 2
+    ent_rows = N * H * 2
+    return {
+        "plan": 2 * N * 4 + N * 4,
+        "dispatch": tok_rows + ent_rows + N * 4,
+        "combine": ent_rows + N * 4 + N * 4 + tok_rows,
+    }
+
+
+def read_peaks() -> tuple[float, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("move_kernels.cu", "plan_kernels.cu", "zb_internal.cuh"):
+        with open(os.path.join(ROOT, "token_dispatch_top_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str) -> float | None:
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the kernels as they are now."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("source_hash") != kernel_source_hash():
+        return None
+    v = rec.get("kernels", {}).get(kernel, {}).get("dram_bytes_per_launch")
+    return float(v) if v is not None else None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while timing."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(parts)
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def oracle_steps(wl, ids, w, hidden_bits, budget_s: float, min_steps: int = 1):
+    """Full CPU-oracle steps (plan + dispatch + combine) until the budget is spent.
+    Returns (steps, seconds)."""
+    import oracle
+    cfg = oracle.Config(wl.P, wl.E, wl.K, wl.S, wl.H, wl.R, wl.C, wl.gpus_per_node, None)
+    buf = np.empty((wl.P, cfg.cap(), wl.H), np.uint16)
+    n = 0
+    t0 = time.perf_counter()
+    while n < min_steps or time.perf_counter() - t0 < budget_s:
+        p = oracle.plan(cfg, ids, want_M=False)
+        oracle.dispatch(cfg, p["dst_row"], hidden_bits, buf)
+        oracle.combine(cfg, p["dst_row"], buf.reshape(-1, wl.H), w)
+        n += 1
+    return n, time.perf_counter() - t0
+
+
+def run_reference(args, wl, rank):
+    """The oracle, as it stands, timed on the host cores."""
+    if rank != 0:
+        return
+    from token_dispatch_top_b200 import synth
+    ids, w = synth.routing(wl, 0)
+    hidden = synth.hidden_bits(wl, 0)
+    oracle_steps(wl, ids, w, hidden, 0.0, min_steps=args.warmup)
+    n, sec = oracle_steps(wl, ids, w, hidden, 0.0, min_steps=args.steps)
+    value = wl.tokens * n / sec
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * sec / n, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_desc(wl), "tokens_per_step": wl.tokens},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{n} full steps of the workload, single-threaded C"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, wl, rank, world, local_rank):
+    import torch
+    from token_dispatch_top_b200 import build, synth, zb
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    build.build()
+    zb.load()
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        dist = dist_mod
+
+    seed = rank
+    ids_np, w_np = synth.routing(wl, seed)
+    hidden_np = synth.hidden_bits(wl, seed)
+    cfg = zb.Config(P=wl.P, E=wl.E, K=wl.K, S=wl.S, H=wl.H, R=wl.R, C=wl.C,
+                    gpus_per_node=wl.gpus_per_node)
+    P, S, K, H, cap = cfg.P, cfg.S, cfg.K, cfg.H, cfg.cap
+
+    ids = torch.from_numpy(ids_np).to(dev)
+    w = torch.from_numpy(w_np).to(dev)
+    hidden = torch.from_numpy(hidden_np.view(np.int16)).to(dev).view(torch.bfloat16)
+    plan = zb.Plan(cfg, dev, with_row_src=False)
+    buf = torch.empty((P, cap, H), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((P, S, H), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        zb.plan(plan, ids)
+        zb.dispatch(plan, hidden, buf)
+        zb.combine(plan, buf, w, out)
+
+    # the plan must balance (status OK) and must fit the S*K buffers
+    step()
+    status, max_load = zb.plan_status(plan)
+    if status < 0:
+        raise RuntimeError(f"plan failed: {zb.strerror(status)}")
+
+    def barrier():
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    barrier()
+    n_ev = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_ev)]
+    with ClockSampler(local_rank) as clocks:
+        barrier()
+        t0 = time.perf_counter()
+        for k in range(args.steps):
+            flush.zero_()
+            ev[k][0].record(stream)
+            zb.plan(plan, ids)
+            ev[k][1].record(stream)
+            zb.dispatch(plan, hidden, buf)
+            ev[k][2].record(stream)
+            zb.combine(plan, buf, w, out)
+            ev[k][3].record(stream)
+        barrier()
+        wall = time.perf_counter() - t0
+    status, _ = zb.plan_status(plan)
+    if status < 0:
+        raise RuntimeError(f"plan failed: {zb.strerror(status)}")
+    t_plan = [ev[k][0].elapsed_time(ev[k][1]) for k in range(n_ev)]
+    t_disp = [ev[k][1].elapsed_time(ev[k][2]) for k in range(n_ev)]
+    t_comb = [ev[k][2].elapsed_time(ev[k][3]) for k in range(n_ev)]
+    step_ms = sum(ev[k][0].elapsed_time(ev[k][3]) for k in range(n_ev))  # total over K steps
+
+    # ---- end to end through the public API, pinned host buffers
+    ids_h = torch.from_numpy(ids_np).pin_memory()
+    w_h = torch.from_numpy(w_np).pin_memory()
+    hid_h = torch.from_numpy(hidden_np.view(np.int16)).pin_memory()
+    out_h = torch.empty((P, S, H), dtype=torch.int16).pin_memory()
+    stats_h = torch.empty((zb.STATS_LEN,), dtype=torch.int64).pin_memory()
+    ids_d = torch.empty_like(ids)
+    w_d = torch.empty_like(w)
+    hid_d = torch.empty((P, S, H), dtype=torch.int16, device=dev)
+
+    def e2e_step():
+        ids_d.copy_(ids_h, non_blocking=True)
+        w_d.copy_(w_h, non_blocking=True)
+        hid_d.copy_(hid_h, non_blocking=True)
+        zb.plan(plan, ids_d)
+        zb.dispatch(plan, hid_d.view(torch.bfloat16), buf)
+        zb.combine(plan, buf, w_d, out)
+        out_h.copy_(out.view(torch.int16), non_blocking=True)
+        stats_h.copy_(plan.stats, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e2e_ms = 0.0
+    for _ in range(args.steps):
+        flush.zero_()
+        e0.record(stream)
+        e2e_step()
+        e1.record(stream)
+        e1.synchronize()
+        if int(stats_h[zb.STAT_STATUS]) < 0:
+            raise RuntimeError("plan failed in the end-to-end loop")
+        e2e_ms += e0.elapsed_time(e1)
+    barrier()
+    h2d = ids_np.nbytes + w_np.nbytes + hidden_np.nbytes
+    d2h = P * S * H * 2 + zb.STATS_LEN * 8
+
+    # ---- max over ranks
+    vals = [step_ms, e2e_ms, sum(t_disp), sum(t_comb), sum(t_plan)]
+    if dist is not None:
+        tt = torch.tensor(vals, dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        vals = tt.tolist()
+    step_ms, e2e_ms, disp_ms, comb_ms, plan_ms = vals
+    if rank != 0:
+        return
+
+    tokens = wl.tokens * world
+    ms_per_step = step_ms / args.steps
+    value = tokens / (ms_per_step / 1000.0)
+    e2e_value = tokens / (e2e_ms / args.steps / 1000.0)
+    ab = algorithmic_bytes(wl)
+    disp_ms_avg = disp_ms / args.steps
+    comb_ms_avg = comb_ms / args.steps
+    dom, dom_ms = ("k_combine", comb_ms_avg) if comb_ms_avg >= disp_ms_avg else \
+        ("k_dispatch", disp_ms_avg)
+    dom_bytes = ab["combine"] if dom == "k_combine" else ab["dispatch"]
+    peak, peak_kind = read_peaks()
+    achieved = dom_bytes / (dom_ms / 1000.0) / 1e9
+    traffic = recorded_traffic(dom)
+
+    cpu = None
+    if world == 1:
+        n, sec = oracle_steps(wl, ids_np, w_np, hidden_np, budget_s=10.0)
+        cpu = {"value": wl.tokens * n / sec, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{n} full steps (plan+dispatch+combine) of the same workload, "
+                         "single-threaded C"}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": workload_desc(wl), "tokens_per_step_per_gpu": wl.tokens,
+                   "accumulate": "f32", "experts": "identity (y = dispatched rows)",
+                   "l2": "flushed before every step by a 256 MB write (outside the timing)",
+                   "parallelism": f"replicas x{world}"},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 5 * args.steps,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "algorithmic_bytes": dom_bytes},
+        "kernels_ms": {"plan": plan_ms / args.steps, "dispatch": disp_ms_avg,
+                       "combine": comb_ms_avg},
+        "kernels_gbs": {"dispatch": ab["dispatch"] / disp_ms_avg / 1e6,
+                        "combine": ab["combine"] / comb_ms_avg / 1e6},
+        "wall_s": wall,
+        "clocks": clocks.summary(),
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be at least 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from token_dispatch_top_b200 import synth
+    wl = synth.WORKLOADS[WORKLOAD]
+
+    if args.impl == "reference":
+        run_reference(args, wl, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+        try:
+            run_ours(args, wl, rank, world, local_rank)
+        finally:
+            dist.destroy_process_group()
+    else:
+        run_ours(args, wl, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

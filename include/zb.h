@@ -1,0 +1,199 @@
+/*
+ * zb.h -- C ABI of libzb: load-balanced MoE token dispatch and combine on one
+ * B200 (sm_100a), with the P expert-parallel ranks virtual and their buffers
+ * partitioned inside one device memory.
+ *
+ * One invocation is five steps, in order:
+ *   1. per-rank, per-expert histogram of the top-K routing ids        (zb_plan)
+ *   2. greedy hot-expert replica planner down to the water level T    (zb_plan)
+ *   3. locality-first assignment of every (token,k), cu_seqlens       (zb_plan)
+ *   4. scatter of bf16 token rows into expert-grouped S*K buffers     (zb_dispatch)
+ *   5. gate-weighted combine gather, fp32 accumulation in k order     (zb_combine)
+ *
+ * Conventions for every entry point:
+ *  - Every pointer argument except `cfg`, `plan` (the struct itself) and the
+ *    out-parameters of zb_plan_status is DEVICE memory owned by the caller.
+ *    The library allocates nothing and keeps no state between calls.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Every call except zb_plan_status only enqueues work on it and
+ *    returns without synchronising.
+ *  - Layouts are dense row-major, C order, no padding.  bf16 arrays are passed
+ *    as uint16_t bit patterns.  Rows and tensors must be 16-byte aligned
+ *    (H % 8 == 0 and 16-byte aligned base pointers).
+ *  - Return value: ZB_OK (0), a positive warning, or a negative error.  A call
+ *    that returns an error has enqueued nothing.  Errors that only the device
+ *    can see (bad ids, capacity) are recorded in plan->stats and reported by
+ *    zb_plan_status; dispatch and combine launched on such a plan do nothing.
+ *
+ * Notation: i = source rank, j = destination rank, e = expert, Eh = E/P home
+ * experts per rank (expert e lives on rank home(e) = e / Eh), f = s*K + k the
+ * flat index of an entry inside its source rank, g = i*S*K + f the global
+ * entry index, cap = cfg->cap_rows.
+ */
+#ifndef ZB_H
+#define ZB_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ZB_API __attribute__((visibility("default")))
+#else
+#define ZB_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------ status codes */
+#define ZB_OK 0
+#define ZB_WARN_UNBALANCED 1 /* R slots did not permit T: some rank ends above T */
+#define ZB_ERR_INVALID (-1)  /* bad configuration, pointer, size or alignment */
+#define ZB_ERR_CAPACITY (-2) /* planned max rank load > cap_rows */
+#define ZB_ERR_BAD_ID (-3)   /* a routing id outside [0, E) */
+#define ZB_ERR_TIMEOUT (-4)  /* reserved: a bounded device wait gave up */
+#define ZB_ERR_CUDA (-5)     /* a CUDA runtime call failed */
+
+/* Problem shape.
+ *   P   ranks, 1..32          E  experts, P..384, E % P == 0
+ *   K   top-K, 1..16          S  tokens per rank, >= 0
+ *   H   hidden width in bf16 elements, H >= 8, H % 8 == 0
+ *   R   replica (helper) slots per rank, 0..P-1
+ *   C   relaxation ratio of the routing constraint |sum_i M_ij - q_j| <= C q_j,
+ *       0 <= C < 1 (validated and recorded; quotas are met exactly, see zb_plan)
+ *   gpus_per_node  1 = flat locality cost; g > 1 groups ranks into nodes of g
+ *       consecutive ranks (P % g == 0)
+ *   cap_rows  rows of each rank's receive buffer, >= S*K; P*cap_rows and
+ *       P*S*K must fit in int32 */
+typedef struct zb_config {
+  int P, E, K, S, H, R;
+  float C;
+  int gpus_per_node;
+  int cap_rows;
+} zb_config;
+
+/* Indices into plan->stats (int64). */
+#define ZB_STAT_STATUS 0        /* final status of the plan (a ZB_* code) */
+#define ZB_STAT_MAX_LOAD 1      /* max_j load_after[j] */
+#define ZB_STAT_N_REPLICAS 2    /* filled helper slots */
+#define ZB_STAT_N_ITERS 3       /* greedy iterations taken */
+#define ZB_STAT_WATER_LEVEL 4   /* T = ceil(sum_r L_r / P) */
+#define ZB_STAT_LOCALITY_COST 5 /* sum_{e,i,j} a_ij M^e_ij */
+#define ZB_STAT_BAD_IDS 6       /* count of ids outside [0, E) */
+#define ZB_STATS_LEN 8
+
+/* The plan: caller-allocated device buffers that zb_plan fills and
+ * zb_dispatch / zb_combine read.  Shapes (int32 unless stated):
+ *   cnt         [P][E]        cnt[i][e] = #{(s,k): ids[i,s,k] = e}
+ *   rep_expert  [P][R]        expert held by helper slot (j, r), -1 = empty
+ *   rep_quota   [P][R]        rows that slot receives (0 if empty)
+ *   home_quota  [E]           rows the home copy of e receives
+ *   load_before [P]           L_j = rows homed on j before planning
+ *   load_after  [P]           rows rank j receives after planning
+ *   cu_seqlens  [P][Eh+R+1]   exclusive prefix of the rows of rank j's groups:
+ *                             groups 0..Eh-1 are its home experts j*Eh+g,
+ *                             groups Eh..Eh+R-1 its helper slots 0..R-1
+ *   dst_row     [P][S][K]     j*cap + row of each entry in the receive buffers
+ *   row_src     [P][cap]      inverse of dst_row: g, or -1 for an unused row;
+ *                             OPTIONAL, may be NULL (then not written)
+ *   stats       int64 [ZB_STATS_LEN], see ZB_STAT_* */
+typedef struct zb_plan_t {
+  int32_t *cnt;
+  int32_t *rep_expert;
+  int32_t *rep_quota;
+  int32_t *home_quota;
+  int32_t *load_before;
+  int32_t *load_after;
+  int32_t *cu_seqlens;
+  int32_t *dst_row;
+  int32_t *row_src;
+  int64_t *stats;
+} zb_plan_t;
+
+/* Text of a status code (static storage; never NULL). */
+ZB_API const char *zb_strerror(int status);
+
+/* ZB_OK if `cfg` satisfies every bound listed at zb_config, else
+ * ZB_ERR_INVALID.  Host only; touches no device. */
+ZB_API int zb_validate(const zb_config *cfg);
+
+/* Bytes of device scratch memory zb_plan needs for `cfg` (0 if `cfg` is
+ * invalid).  Host only.  The workspace holds the per-chunk histograms, the
+ * per-(source, expert) segment table and error flags; its contents need not
+ * be initialised and are dead after the plan's kernels complete. */
+ZB_API size_t zb_workspace_bytes(const zb_config *cfg);
+
+/* Steps 1-3: histogram, greedy replica plan, assignment.
+ *
+ * Steps, after the pages:
+ *  - count routes per rank and expert (ISER-MoE, Methodology, HALO-Q
+ *    Scheduler, stage 1, where ranks share these counts);
+ *  - water level T = ceil(sum_r L_r / P) (ISER-MoE, HALO-Q Objective 1); since
+ *    every entry routes exactly once, T = S*K, MoonEP's per-rank S x K
+ *    invariant ("What MoonEP enforces and how");
+ *  - greedy placement: while the busiest rank d (ties: lowest rank) is above T,
+ *    it offers its heaviest home expert (largest remaining home quota, ties:
+ *    lowest expert) for which an eligible receiver exists; eligible = another
+ *    rank with a free slot, load below T and no copy of the expert; the
+ *    receiver is the one whose node does not yet hold the expert, then the
+ *    lowest load, then the lowest rank (Zepp "4.1 Expert Placement and Token
+ *    Routing": R extra slots per GPU, round-robin across nodes first); it takes
+ *    m = min(load_d - T, T - load_r, quota_e) rows into its lowest free slot
+ *    (HALO-Q stages 2-3).  A donor with no movable expert is marked stuck;
+ *  - routing: expert e's rows are assigned to its hosts by eq. (1) of Zepp 4.1,
+ *    minimising sum a_ij M^e_ij with each host receiving exactly its quota
+ *    (a_ij = 0 same rank, 1 other rank; with nodes 1 same node, 4 other node):
+ *    each host first serves its own rank, then per cost level, hosts in
+ *    ascending rank take from sources in ascending rank (HALO-Q stage 5,
+ *    the route rewrite that keeps rows local before moving them);
+ *  - rows: source i walks its entries of expert e in flat order and fills its
+ *    hosts in order of (a_ij, j); inside a group, rows are ordered by source
+ *    rank, then flat index; cu_seqlens indexes the groups (MoonEP, section on
+ *    what it enforces: the on-GPU planner hands kernels these offsets).
+ *
+ * topk_ids: device int32 [P][S][K].  plan: all required buffers as listed at
+ * zb_plan_t.  workspace: device, zb_workspace_bytes(cfg) bytes (pass that
+ * count as workspace_bytes), 256-byte aligned.
+ * Returns ZB_OK once the work is enqueued, ZB_ERR_INVALID (bad cfg, NULL
+ * buffer, short workspace) or ZB_ERR_CUDA.  The plan's own outcome (OK,
+ * UNBALANCED, CAPACITY, BAD_ID) lands in plan->stats; read it with
+ * zb_plan_status.  On CAPACITY or BAD_ID, dst_row and row_src are undefined. */
+ZB_API int zb_plan(const zb_config *cfg, const int32_t *topk_ids, const zb_plan_t *plan,
+            void *workspace, size_t workspace_bytes, void *stream);
+
+/* Synchronises `stream`, then returns the plan's status (ZB_OK,
+ * ZB_WARN_UNBALANCED, ZB_ERR_CAPACITY, ZB_ERR_BAD_ID), or ZB_ERR_CUDA.
+ * If max_load is not NULL it receives the planned max rank load (host int). */
+ZB_API int zb_plan_status(const zb_config *cfg, const zb_plan_t *plan, void *stream,
+                   int32_t *max_load);
+
+/* Step 4: buf[dst_row[i,s,k]][:] = hidden[i,s][:], bit for bit: each token row
+ * is written into the fixed-shape, expert-grouped receive buffer of every rank
+ * that serves one of its K experts (MoonEP, section on what it enforces: rows
+ * go straight into static per-rank buffers with no staging copy; on one GPU
+ * that remote write is a local scatter).  hidden: device bf16 [P][S][H]; buf: device bf16 [P][cap][H].
+ * Rows of buf past load_after[j] are not written.  If plan->stats holds an
+ * error status the kernel writes nothing.  Returns ZB_OK, ZB_ERR_INVALID or
+ * ZB_ERR_CUDA. */
+ZB_API int zb_dispatch(const zb_config *cfg, const zb_plan_t *plan, const uint16_t *hidden,
+                uint16_t *buf, void *stream);
+
+/* Step 5: for every token t = (i,s) and column h,
+ *   acc = +0.0f;  for k = 0..K-1: acc = fmaf(w[t][k], float(y[dst_row[t][k]][h]), acc);
+ *   out[t][h] = bf16(acc), rounded to nearest, ties to even,
+ * the inverse of dispatch weighted by the gates (Zepp 4.2, merge for combine;
+ * ISER-MoE, Key Formula, the combine half of the dispatch+combine traffic).  One
+ * rounding per term, in this fixed order, so the result is reproducible bit
+ * for bit.  y: device bf16 [P][cap][H] (expert outputs, same layout as buf);
+ * topk_weights: device float32 [P][S][K]; out: device bf16 [P][S][H].  If
+ * plan->stats holds an error status the kernel writes nothing.  Returns
+ * ZB_OK, ZB_ERR_INVALID or ZB_ERR_CUDA. */
+ZB_API int zb_combine(const zb_config *cfg, const zb_plan_t *plan, const uint16_t *y,
+               const float *topk_weights, uint16_t *out, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZB_H */

@@ -1,0 +1,103 @@
+"""The C ABI without a GPU: the library builds, loads, exports every entry
+point include/zb.h declares, and its host-side logic (validation, workspace
+sizing, status text, argument checks) behaves as documented.  No call here
+touches a device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+from token_dispatch_top_b200 import build, zb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return zb.load()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "zb.h")).read()
+    return sorted(set(re.findall(r"ZB_API\s+[\w\s\*]*?\b(zb_\w+)\s*\(", text)))
+
+
+def test_exports_match_header(lib):
+    declared = _declared()
+    assert set(declared) >= set(zb.EXPORTS)
+    out = subprocess.check_output(["nm", "-D", "--defined-only", zb.LIB_PATH], text=True)
+    exported = sorted(line.split()[-1] for line in out.splitlines()
+                      if line.split()[-1].startswith("zb_"))
+    assert exported == declared
+    for name in declared:
+        assert hasattr(lib, name)
+
+
+def test_strerror(lib):
+    for code in (zb.OK, zb.WARN_UNBALANCED, zb.ERR_INVALID, zb.ERR_CAPACITY, zb.ERR_BAD_ID,
+                 zb.ERR_TIMEOUT, zb.ERR_CUDA, 12345):
+        assert isinstance(zb.strerror(code), str) and zb.strerror(code)
+    assert zb.strerror(12345) == "unknown status"
+
+
+def _both(**kw):
+    base = dict(P=4, E=16, K=2, S=64, H=128, R=1, C=0.1, gpus_per_node=1, cap_rows=None)
+    base.update(kw)
+    return zb.Config(**base), oracle.Config(**base)
+
+
+@pytest.mark.parametrize("kw", [
+    {}, dict(P=0), dict(P=33), dict(E=15), dict(E=400), dict(E=2, P=4), dict(K=0), dict(K=17),
+    dict(S=-1), dict(S=0), dict(H=0), dict(H=4), dict(H=12), dict(R=-1), dict(R=4), dict(R=3),
+    dict(C=-0.5), dict(C=1.0), dict(C=0.99), dict(gpus_per_node=0), dict(gpus_per_node=3),
+    dict(gpus_per_node=2), dict(cap_rows=127), dict(cap_rows=128), dict(P=32, E=384, R=31),
+    dict(P=1, E=384, R=0), dict(K=16), dict(S=2 ** 27, K=16), dict(S=2 ** 26, K=8, P=8, E=16),
+])
+def test_validation_agrees_with_oracle(lib, kw):
+    c, o = _both(**kw)
+    assert zb.validate(c) == oracle.validate(o), kw
+
+
+def test_workspace_bytes(lib):
+    c, _ = _both()
+    n = zb.workspace_bytes(c)
+    assert n > 0 and n % 256 == 0
+    # grows with the number of chunks
+    c2, _ = _both(S=64 * 1024)
+    assert zb.workspace_bytes(c2) > n
+    bad, _ = _both(P=0)
+    assert zb.workspace_bytes(bad) == 0
+
+
+def test_entry_points_reject_bad_arguments_without_a_device(lib):
+    cfg = zb.Config(P=4, E=16, K=2, S=64, H=128, R=1).c()
+    plan = zb._Plan()  # all NULL
+    # NULL plan buffers / workspace -> invalid, nothing enqueued
+    assert lib.zb_plan(ctypes.byref(cfg), None, ctypes.byref(plan), None, 0, None) == \
+        zb.ERR_INVALID
+    assert lib.zb_dispatch(ctypes.byref(cfg), ctypes.byref(plan), None, None, None) == \
+        zb.ERR_INVALID
+    assert lib.zb_combine(ctypes.byref(cfg), ctypes.byref(plan), None, None, None, None) == \
+        zb.ERR_INVALID
+    assert lib.zb_plan_status(ctypes.byref(cfg), ctypes.byref(plan), None, None) == \
+        zb.ERR_INVALID
+    bad = zb.Config(P=4, E=15, K=2, S=64, H=128, R=1).c()
+    assert lib.zb_plan(ctypes.byref(bad), None, ctypes.byref(plan), None, 0, None) == \
+        zb.ERR_INVALID
+    # misaligned rows are refused before any launch
+    fake = zb._Plan(*([16] * 10))
+    assert lib.zb_dispatch(ctypes.byref(cfg), ctypes.byref(fake), 8, 16, None) == \
+        zb.ERR_INVALID
+    assert lib.zb_combine(ctypes.byref(cfg), ctypes.byref(fake), 16, 16, 8, None) == \
+        zb.ERR_INVALID
+    # a short or misaligned workspace is refused
+    ws = zb.workspace_bytes(zb.Config(P=4, E=16, K=2, S=64, H=128, R=1))
+    assert lib.zb_plan(ctypes.byref(cfg), 16, ctypes.byref(fake), 256, ws - 1, None) == \
+        zb.ERR_INVALID
+    assert lib.zb_plan(ctypes.byref(cfg), 16, ctypes.byref(fake), 128, ws, None) == \
+        zb.ERR_INVALID

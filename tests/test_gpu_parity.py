@@ -1,0 +1,368 @@
+"""GPU parity: the sm_100a path through the C ABI against the CPU oracle.
+
+Bit-exact for the histogram, plan tables, cu_seqlens, dst_row/row_src, the
+dispatched rows and the combined output (the combine's summation order is
+fixed, so no tolerance is taken).  Small cases compare every element; the
+full-size workloads compare the whole plan and sampled rows of dispatch and
+combine, plus properties that hold at any size.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import parity
+from parity import bf16_to_bits, bits_to_bf16, cfgs, gpu_plan, plan_tables, assert_plan_equal
+from token_dispatch_top_b200 import build, synth, zb
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_examples.json")
+
+
+@pytest.fixture(scope="module")
+def dev(cuda_device):
+    build.build()
+    zb.load()
+    return cuda_device
+
+
+def _rand_bits(rng, shape):
+    x = rng.standard_normal(shape, dtype=np.float32)
+    return torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def full_parity(zc, oc, ids, w, hidden_bits, y_bits, dev, with_row_src=True, stream=None):
+    """Plan, dispatch and combine on both sides; compare every element."""
+    ctx = torch.cuda.stream(stream) if stream is not None else torch.cuda.stream(
+        torch.cuda.current_stream())
+    with ctx:
+        p, status, max_load = gpu_plan(zc, ids, dev, with_row_src)
+        g = plan_tables(p)
+    o = oracle.plan(oc, ids)
+    assert_plan_equal(g, o, status)
+    if status < 0:
+        return p, status
+    P, S, K, H, cap = zc.P, zc.S, zc.K, zc.H, zc.cap
+    with ctx:
+        hid = bits_to_bf16(hidden_bits, dev)
+        buf = torch.full((P, cap, H), 0, dtype=torch.int16, device=dev)
+        buf.fill_(parity.SENTINEL)
+        buf = buf.view(torch.bfloat16)
+        zb.dispatch(p, hid, buf)
+        w_d = torch.from_numpy(np.ascontiguousarray(w, np.float32)).to(dev)
+        out_a = torch.empty((P, S, H), dtype=torch.bfloat16, device=dev)
+        zb.combine(p, buf, w_d, out_a)
+        y_d = bits_to_bf16(y_bits, dev).view(P, cap, H)
+        out_b = torch.empty((P, S, H), dtype=torch.bfloat16, device=dev)
+        zb.combine(p, y_d, w_d, out_b)
+        torch.cuda.current_stream().synchronize()
+    ob = np.full((P, cap, H), parity.SENTINEL, np.uint16)
+    oracle.dispatch(oc, o["dst_row"], hidden_bits, ob)
+    gb = bf16_to_bits(buf)
+    np.testing.assert_array_equal(gb, ob)  # rows past the load keep the sentinel too
+    oa = oracle.combine(oc, o["dst_row"], ob.reshape(P * cap, H), w)
+    np.testing.assert_array_equal(bf16_to_bits(out_a), oa)
+    oy = oracle.combine(oc, o["dst_row"], y_bits.reshape(P * cap, H), w)
+    np.testing.assert_array_equal(bf16_to_bits(out_b), oy)
+    return p, status
+
+
+# ------------------------------------------------------------- hand examples
+
+@pytest.mark.parametrize("ex", json.load(open(GOLDEN))["examples"], ids=lambda e: e["name"])
+def test_hand_examples(dev, ex):
+    d = ex["cfg"]
+    kw = dict(P=d["P"], E=d["E"], K=d["K"], S=d["S"], H=d["H"], R=d["R"],
+              gpus_per_node=d.get("gpus_per_node", 1), cap_rows=d.get("cap_rows"))
+    zc, oc = zb.Config(**kw), oracle.Config(**kw)
+    ids = np.array(ex["ids"], np.int32).reshape(zc.P, zc.S, zc.K)
+    rng = np.random.default_rng(0)
+    w = rng.dirichlet(np.ones(zc.K), size=(zc.P, zc.S)).astype(np.float32)
+    full_parity(zc, oc, ids, w, _rand_bits(rng, (zc.P, zc.S, zc.H)),
+                _rand_bits(rng, (zc.P * zc.cap, zc.H)), dev)
+
+
+# ------------------------------------------------------------- random small
+
+def _small_cases(n=60, seed=21):
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(n):
+        P = int(rng.choice([1, 2, 3, 4, 6, 8, 16, 32]))
+        gpn = int(rng.choice([g for g in (1, 2, 4, 8) if P % g == 0]))
+        Eh = int(rng.integers(1, min(12, 384 // P) + 1))
+        E = P * Eh
+        K = int(rng.integers(1, 9))
+        S = int(rng.integers(0, 300))
+        R = int(rng.integers(0, min(P, 4)))
+        H = int(rng.choice([8, 16, 64, 136]))
+        p = 1.0 / np.arange(1, E + 1) ** rng.uniform(0, 2)
+        p = p[rng.permutation(E)] / p.sum()
+        ids = rng.choice(E, size=(P, S, K), p=p).astype(np.int32)
+        out.append((dict(P=P, E=E, K=K, S=S, H=H, R=R, C=0.1, gpus_per_node=gpn), ids))
+    return out
+
+
+SMALL = _small_cases()
+
+
+@pytest.mark.parametrize("k", range(len(SMALL)))
+def test_random_small(dev, k):
+    kw, ids = SMALL[k]
+    rng = np.random.default_rng(1000 + k)
+    # cap large enough for an unbalanced plan: the sum of all entries
+    kw = dict(kw, cap_rows=max(1, kw["P"] * kw["S"] * kw["K"]))
+    zc, oc = zb.Config(**kw), oracle.Config(**kw)
+    w = rng.dirichlet(np.ones(zc.K), size=(zc.P, zc.S)).astype(np.float32)
+    full_parity(zc, oc, ids, w, _rand_bits(rng, (zc.P, zc.S, zc.H)),
+                _rand_bits(rng, (zc.P * zc.cap, zc.H)), dev)
+
+
+# ------------------------------------------------------------- named workloads
+
+@pytest.mark.parametrize("name,seed", [("tiny", 0), ("tiny", 1), ("mid", 0), ("mid", 1)])
+def test_workload_full(dev, name, seed):
+    """tiny and mid (the benchmark workload, same launch configuration) compared
+    element by element, including the receive buffers."""
+    wl = synth.WORKLOADS[name]
+    zc, oc = cfgs(wl)
+    ids, w = synth.routing(wl, seed)
+    hidden = synth.hidden_bits(wl, seed)
+    y = synth.y_bits(wl, zc.P * zc.cap, seed)
+    p, status = full_parity(zc, oc, ids, w, hidden, y, dev, with_row_src=(name == "tiny"))
+    assert status == oracle.OK  # both balance to T = S*K
+
+
+@pytest.mark.parametrize("seed", [2, 3, 4, 5])
+def test_mid_seed_sweep_plan(dev, seed):
+    wl = synth.WORKLOADS["mid"]
+    zc, oc = cfgs(wl)
+    ids, _ = synth.routing(wl, seed)
+    p, status, _ = gpu_plan(zc, ids, dev)
+    assert_plan_equal(plan_tables(p), oracle.plan(oc, ids), status)
+
+
+def sampled_data_parity(zc, oc, p, o, ids, w, hidden_d, dev, n=384, seed=0):
+    """Dispatch and combine on the device at full size; compare sampled token
+    rows with the oracle computed one token at a time."""
+    P, S, K, H, cap = zc.P, zc.S, zc.K, zc.H, zc.cap
+    rng = np.random.default_rng(seed)
+    tok = np.unique(np.concatenate([[0, P * S - 1], rng.integers(0, P * S, n)]))
+    buf = torch.empty((P, cap, H), dtype=torch.int16, device=dev)
+    buf.fill_(parity.SENTINEL)
+    buf = buf.view(torch.bfloat16)
+    zb.dispatch(p, hidden_d, buf)
+    # sampled rows: every destination row of a sampled token holds its hidden row
+    dst = o["dst_row"].reshape(P * S, K)
+    rows = torch.from_numpy(dst[tok].ravel().astype(np.int64)).to(dev)
+    got = buf.view(P * cap, H).index_select(0, rows).view(len(tok), K, H)
+    want = hidden_d.view(P * S, H).index_select(0, torch.from_numpy(tok).to(dev))
+    assert torch.equal(got.view(torch.int16), want.view(torch.int16)[:, None, :].expand_as(
+        got.view(torch.int16)))
+    # rows past each rank's load are untouched
+    la = o["load_after"]
+    spare = [(j, r) for j in range(P) for r in rng.integers(la[j], cap, 8) if la[j] < cap]
+    if spare:
+        idx = torch.tensor([j * cap + r for j, r in spare], device=dev)
+        assert bool((buf.view(P * cap, H).index_select(0, idx).view(torch.int16) ==
+                     parity.SENTINEL).all())
+    # property at full size: y = buf and weights summing to 1 give back each
+    # token's row within one bf16 ulp
+    w_d = torch.from_numpy(np.ascontiguousarray(w)).to(dev)
+    out = torch.empty((P, S, H), dtype=torch.bfloat16, device=dev)
+    zb.combine(p, buf, w_d, out)
+    diff = (out.float() - hidden_d.float()).abs()
+    ulp = torch.where(hidden_d.float() == 0, torch.full_like(diff, 1e-38),
+                      hidden_d.float().abs() * 2.0 ** -7)
+    assert bool((diff <= ulp).all())
+    # independent expert outputs: exact against the oracle on sampled tokens
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234 + seed)
+    y = torch.randn((P, cap, H), generator=gen, device=dev, dtype=torch.bfloat16)
+    zb.combine(p, y, w_d, out)
+    yk = bf16_to_bits(y.view(P * cap, H).index_select(0, rows))
+    n_t = len(tok)
+    ocfg = oracle.Config(P=1, E=1, K=K, S=n_t, H=H, R=0, cap_rows=n_t * K)
+    want_o = oracle.combine(ocfg, np.arange(n_t * K, dtype=np.int32).reshape(1, n_t, K), yk,
+                            w.reshape(P * S, K)[tok].reshape(1, n_t, K))
+    got_o = bf16_to_bits(out.view(P * S, H).index_select(0, torch.from_numpy(tok).to(dev)))
+    np.testing.assert_array_equal(got_o, want_o[0])
+    del buf, y, out
+
+
+@pytest.mark.parametrize("name", ["hot", "hier"])
+def test_workload_full_size(dev, name):
+    """Full-size plan bit-exact; dispatch/combine sampled (same launch path)."""
+    wl = synth.WORKLOADS[name]
+    zc, oc = cfgs(wl, cap_rows=2 * wl.S * wl.K)
+    ids, w = synth.routing(wl, 0)
+    p, status, _ = gpu_plan(zc, ids, dev)
+    o = oracle.plan(oc, ids)
+    assert_plan_equal(plan_tables(p), o, status)
+    assert status in (oracle.OK, oracle.UNBALANCED)
+    hidden = synth.hidden_device(wl, 0, 0, dev)
+    sampled_data_parity(zc, oc, p, o, ids, w, hidden, dev)
+    # at the water level the plan refuses to fit in S*K rows when unbalanced
+    if status == oracle.UNBALANCED:
+        zc2, oc2 = cfgs(wl)
+        p2, st2, _ = gpu_plan(zc2, ids, dev)
+        assert st2 == oracle.ERR_CAPACITY == oracle.plan(oc2, ids, want_M=False)["status"]
+    torch.cuda.empty_cache()
+
+
+def test_drift_all_steps(dev):
+    """64 re-planned invocations of the drifting workload: every plan bit-exact,
+    dispatch/combine sampled on a few steps."""
+    wl = synth.WORKLOADS["drift"]
+    zc, oc = cfgs(wl, cap_rows=2 * wl.S * wl.K)
+    data_steps = {0, 1, 32, 63}
+    for step in range(wl.steps):
+        ids, w = synth.routing(wl, 0, step)
+        p, status, _ = gpu_plan(zc, ids, dev, with_row_src=False)
+        o = oracle.plan(oc, ids, want_M=False)
+        assert_plan_equal(plan_tables(p), o, status)
+        if step in data_steps:
+            hidden = synth.hidden_device(wl, 0, step, dev)
+            sampled_data_parity(zc, oc, p, o, ids, w, hidden, dev, n=128, seed=step)
+            del hidden
+            torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------- edge cases
+
+def _run_small(dev, ids, K=None, H=16, R=1, P=None, E=None, cap_rows=None, gpn=1, seed=0,
+               with_row_src=True, stream=None):
+    P = P or ids.shape[0]
+    S = ids.shape[1]
+    K = K or ids.shape[2]
+    kw = dict(P=P, E=E, K=K, S=S, H=H, R=R, C=0.0, gpus_per_node=gpn, cap_rows=cap_rows)
+    zc, oc = zb.Config(**kw), oracle.Config(**kw)
+    rng = np.random.default_rng(seed)
+    w = rng.dirichlet(np.ones(K), size=(P, S)).astype(np.float32)
+    return full_parity(zc, oc, ids, w, _rand_bits(rng, (P, S, H)),
+                       _rand_bits(rng, (P * zc.cap, H)), dev, with_row_src, stream)
+
+
+def test_empty_input(dev):
+    p, status = _run_small(dev, np.zeros((4, 0, 2), np.int32), E=8)
+    assert status == oracle.OK
+
+
+def test_single_rank_and_no_slots(dev):
+    rng = np.random.default_rng(2)
+    _run_small(dev, rng.integers(0, 8, (1, 100, 3)).astype(np.int32), E=8, R=0)
+    _run_small(dev, rng.integers(0, 8, (4, 100, 3)).astype(np.int32), E=8, R=0,
+               cap_rows=1200)
+
+
+def test_ragged_chunks_and_k1(dev):
+    rng = np.random.default_rng(3)
+    # S*K = 3000: one full chunk of 2048 entries and a ragged tail
+    _run_small(dev, rng.integers(0, 9, (3, 1000, 3)).astype(np.int32), E=9, R=2,
+               cap_rows=9000)
+    _run_small(dev, rng.integers(0, 12, (4, 2049, 1)).astype(np.int32), E=12, R=3, H=8,
+               cap_rows=8196)
+
+
+def test_maximum_shape(dev):
+    """P = 32 ranks, E = 384 experts, K = 16, R = 31 slots, two-level cost."""
+    rng = np.random.default_rng(4)
+    P, E, K, S = 32, 384, 16, 96
+    p = 1.0 / np.arange(1, E + 1) ** 1.2
+    ids = np.stack([np.stack([rng.choice(E, K, replace=False, p=p / p.sum())
+                              for _ in range(S)]) for _ in range(P)]).astype(np.int32)
+    _run_small(dev, ids, E=E, R=31, H=64, gpn=8, cap_rows=S * K * 2)
+    _run_small(dev, ids, E=E, R=2, H=64, gpn=1, cap_rows=S * K * P)
+
+
+def test_all_rows_on_one_expert_and_duplicates(dev):
+    _run_small(dev, np.zeros((8, 64, 4), np.int32), E=16, R=7)
+    rng = np.random.default_rng(5)
+    ids = rng.integers(0, 2, (4, 50, 6)).astype(np.int32)  # many duplicates per token
+    _run_small(dev, ids, E=8, R=3, cap_rows=1200)
+
+
+def test_bad_ids_write_nothing(dev):
+    ids = np.zeros((2, 4, 2), np.int32)
+    ids[0, 1, 1] = -1
+    ids[1, 3, 0] = 4
+    zc = zb.Config(P=2, E=4, K=2, S=4, H=16, R=1)
+    p, status, _ = gpu_plan(zc, ids, dev)
+    assert status == oracle.ERR_BAD_ID == oracle.plan(oracle.Config(P=2, E=4, K=2, S=4, H=16,
+                                                                      R=1), ids)["status"]
+    assert int(p.stats[zb.STAT_BAD_IDS]) == 2
+    hid = torch.randn((2, 4, 16), device=dev).to(torch.bfloat16)
+    buf = torch.full((2, 8, 16), parity.SENTINEL, dtype=torch.int16, device=dev) \
+        .view(torch.bfloat16)
+    zb.dispatch(p, hid, buf)
+    out = torch.full((2, 4, 16), parity.SENTINEL, dtype=torch.int16, device=dev) \
+        .view(torch.bfloat16)
+    zb.combine(p, buf, torch.ones((2, 4, 2), device=dev), out)
+    torch.cuda.synchronize()
+    assert bool((buf.view(torch.int16) == parity.SENTINEL).all())
+    assert bool((out.view(torch.int16) == parity.SENTINEL).all())
+
+
+def test_capacity_then_unbalanced(dev):
+    ids = np.array([[0, 1, 2], [0, 1, 2]], np.int32).reshape(2, 3, 1)
+    zc = zb.Config(P=2, E=6, K=1, S=3, H=16, R=1, cap_rows=3)
+    p, status, max_load = gpu_plan(zc, ids, dev)
+    assert status == oracle.ERR_CAPACITY and max_load == 4
+    buf = torch.full((2, 3, 16), parity.SENTINEL, dtype=torch.int16, device=dev) \
+        .view(torch.bfloat16)
+    zb.dispatch(p, torch.randn((2, 3, 16), device=dev).to(torch.bfloat16), buf)
+    torch.cuda.synchronize()
+    assert bool((buf.view(torch.int16) == parity.SENTINEL).all())
+    p, status = _run_small(dev, ids, E=6, R=1, cap_rows=4)
+    assert status == oracle.UNBALANCED
+
+
+def test_without_row_src_and_on_a_side_stream(dev):
+    rng = np.random.default_rng(6)
+    ids = rng.integers(0, 16, (4, 300, 2)).astype(np.int32)
+    side = torch.cuda.Stream()
+    _run_small(dev, ids, E=16, R=2, cap_rows=2400, with_row_src=False, stream=side)
+
+
+def test_plan_buffers_are_reusable(dev):
+    """A second plan into the same buffers leaves no trace of the first."""
+    wl = synth.WORKLOADS["tiny"]
+    zc, oc = cfgs(wl)
+    p = zb.Plan(zc, dev)
+    for seed in (0, 1, 2):
+        ids, _ = synth.routing(wl, seed)
+        zb.plan(p, torch.from_numpy(ids).to(dev))
+        status, _ = zb.plan_status(p)
+        assert_plan_equal(plan_tables(p), oracle.plan(oc, ids), status)
+
+
+def test_combine_special_values(dev):
+    """Infinities, subnormals and signed zeros follow IEEE through the fold;
+    NaN stays NaN (its payload is not compared)."""
+    P, S, K, H = 2, 8, 3, 64
+    rng = np.random.default_rng(7)
+    ids = rng.integers(0, 4, (P, S, K)).astype(np.int32)
+    kw = dict(P=P, E=4, K=K, S=S, H=H, R=1, cap_rows=P * S * K)
+    zc, oc = zb.Config(**kw), oracle.Config(**kw)
+    p, status, _ = gpu_plan(zc, ids, dev)
+    o = oracle.plan(oc, ids)
+    assert status >= 0
+    y = _rand_bits(rng, (P * zc.cap, H))
+    specials = np.array([0x7F80, 0xFF80, 0x7FC0, 0x0001, 0x8001, 0x8000, 0x0000, 0x7F7F],
+                        np.uint16)
+    y.ravel()[rng.integers(0, y.size, 400)] = rng.choice(specials, 400)
+    w = rng.standard_normal((P, S, K)).astype(np.float32)
+    w.ravel()[:5] = [0.0, -0.0, 1e-40, 3e38, -3e38]
+    out = torch.empty((P, S, H), dtype=torch.bfloat16, device=dev)
+    zb.combine(p, bits_to_bf16(y, dev).view(P, zc.cap, H),
+               torch.from_numpy(w).to(dev), out)
+    got = bf16_to_bits(out)
+    want = oracle.combine(oc, o["dst_row"], y, w)
+    nan_g = ((got & 0x7F80) == 0x7F80) & ((got & 0x7F) != 0)
+    nan_w = ((want & 0x7F80) == 0x7F80) & ((want & 0x7F) != 0)
+    np.testing.assert_array_equal(nan_g, nan_w)
+    np.testing.assert_array_equal(got[~nan_w], want[~nan_w])

@@ -1,0 +1,523 @@
+// plan_kernels.cu -- steps 1-3 of an invocation on one GPU:
+//   k_hist     per-(source rank, chunk) expert histogram in shared memory
+//   k_planner  one CTA: water level, greedy replica placement (one warp, lanes
+//              = ranks), quotas, cu_seqlens, locality-first transport and the
+//              per-(source, expert) segment table
+//   k_assign   per-(source rank, chunk): stable rank of every entry among the
+//              source's entries of the same expert, then its destination row
+//
+// Sources: ISER-MoE "Methodology / HALO-Q Scheduler" (Objective 1 water level,
+// stages 1, 2, 3, 5); Zepp "4.1 Expert Placement and Token Routing" (R slots
+// per GPU, node-first placement, eq. (1)); MoonEP "What MoonEP enforces and
+// how" (S x K per rank, cu_seqlens, expert-grouped fixed buffers).
+#include "zb_internal.cuh"
+
+namespace zb {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ int warp_sum(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+__device__ __forceinline__ long long warp_sum64(long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    unsigned long long u = __shfl_xor_sync(kFull, v, o);
+    v = u > v ? u : v;
+  }
+  return v;
+}
+__device__ __forceinline__ unsigned long long warp_min_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    unsigned long long u = __shfl_xor_sync(kFull, v, o);
+    v = u < v ? u : v;
+  }
+  return v;
+}
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int u = __shfl_up_sync(kFull, v, o);
+    if (lane >= o) v += u;
+  }
+  return v;
+}
+
+// a_ij of eq. (1): 0 same rank; 1 other rank (flat) or same node; 4 other node.
+__device__ __forceinline__ int cost_a(int i, int j, int gpn) {
+  if (i == j) return 0;
+  if (gpn > 1 && (i / gpn) != (j / gpn)) return 4;
+  return 1;
+}
+
+// ------------------------------------------------------------------ step 1
+
+__global__ void __launch_bounds__(kChunkThreads) k_hist(PlanArgs a) {
+  __shared__ int32_t sh[kMaxE];
+  const int c = blockIdx.x, i = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
+  for (int e = tid; e < a.E; e += kChunkThreads) sh[e] = 0;
+  __syncthreads();
+  const int64_t nk = int64_t(a.S) * a.K;
+  const int64_t start = int64_t(c) * kChunk;
+  const int n = (nk - start) < kChunk ? int(nk - start) : kChunk;
+  const int32_t* src = a.ids + int64_t(i) * nk + start;
+  int bad = 0;
+  for (int t0 = 0; t0 < n; t0 += kChunkThreads) {  // warp-uniform trip count
+    const int t = t0 + tid;
+    const bool valid = t < n;
+    const int e = valid ? __ldg(src + t) : -1;
+    const bool ok = valid && e >= 0 && e < a.E;
+    bad += (valid && !ok);
+    const unsigned peers = __match_any_sync(kFull, ok ? e : -1);
+    if (ok && lane == __ffs(peers) - 1) atomicAdd(&sh[e], __popc(peers));
+  }
+  bad = warp_sum(bad);
+  if (lane == 0 && bad) atomicAdd(&a.flags[kFlagBadIds], bad);
+  __syncthreads();
+  int32_t* out = a.chunk_hist + (int64_t(i) * a.nchunk + c) * a.E;
+  for (int e = tid; e < a.E; e += kChunkThreads) {
+    const int v = sh[e];
+    out[e] = v;
+    if (v) atomicAdd(&a.cnt[i * a.E + e], v);
+  }
+}
+
+// ------------------------------------------------------------------ step 2+3
+
+struct PlannerSmem {
+  int32_t* cnt;    // [P*E]
+  int32_t* hq;     // [E]   remaining home quota
+  uint32_t* hold;  // [E]   ranks holding a replica of e (bit r)
+  int32_t* repe;   // [P*R]
+  int32_t* repq;   // [P*R]
+  int32_t* cu;     // [P*(Eh+R+1)]
+  int32_t* hoff;   // [E+1]
+  int32_t* M;      // [warps][32 hosts][32 sources]
+  int32_t* q;      // [warps][32 hosts] remaining quota in transport
+  int32_t* misc;   // [16]
+};
+
+__device__ PlannerSmem carve(char* base, const PlanArgs& a) {
+  PlannerSmem s;
+  int32_t* p = reinterpret_cast<int32_t*>(base);
+  s.cnt = p; p += a.P * a.E;
+  s.hq = p; p += a.E;
+  s.hold = reinterpret_cast<uint32_t*>(p); p += a.E;
+  s.repe = p; p += a.P * a.R;
+  s.repq = p; p += a.P * a.R;
+  s.cu = p; p += a.P * (a.Eh + a.R + 1);
+  s.hoff = p; p += a.E + 1;
+  s.q = p; p += kPlanWarps * 32;
+  s.misc = p; p += 16;
+  s.M = p;
+  return s;
+}
+
+enum { kMiscT = 0, kMiscMax = 1, kMiscNrep = 2, kMiscIters = 3, kMiscStatus = 4, kMiscErr = 5 };
+
+// Greedy replica placement, run by one warp; lane r holds rank r's load,
+// filled-slot count and stuck flag.  (ISER-MoE HALO-Q Objective 1 and stages
+// 2-3; Zepp 4.1 R slots per GPU and node-first hierarchical placement.)
+__device__ void greedy_warp(const PlanArgs& a, PlannerSmem& s, int T, int lane) {
+  const int P = a.P, R = a.R, Eh = a.Eh, gpn = a.gpn;
+  int load = 0;
+  if (lane < P) {
+    for (int e = lane * Eh; e < (lane + 1) * Eh; ++e) load += s.hq[e];
+  }
+  int nfill = 0;
+  bool stuck = lane >= P;
+  int iters = 0;
+  const int max_iters = P * R + P + 1;
+  // mask of the ranks on lane's node
+  const unsigned node_mask =
+      gpn >= 32 ? kFull : (((1u << gpn) - 1u) << ((lane / gpn) * gpn));
+  for (int guard = 0; guard <= max_iters; ++guard) {
+    // donor: the busiest non-stuck rank, ties to the lowest rank
+    const unsigned long long dkey =
+        stuck ? 0ull : ((unsigned long long)(unsigned)(load + 1) << 5) | unsigned(31 - lane);
+    const unsigned long long dbest = warp_max_u64(dkey);
+    if (dbest == 0ull) break;
+    const int d = 31 - int(dbest & 31u);
+    const int dload = int(dbest >> 5) - 1;
+    if (dload <= T) break;
+    ++iters;
+    // receivers with room: not the donor, a free slot, load below T
+    const unsigned base = __ballot_sync(kFull, lane < P && lane != d && nfill < R && load < T);
+    // heaviest home expert of d (largest remaining quota, ties: lowest id)
+    // that has an eligible receiver, i.e. a rank in base without a copy
+    unsigned long long ebest = 0ull;
+    for (int x = lane; x < Eh; x += 32) {
+      const int e = d * Eh + x;
+      const int q = s.hq[e];
+      if (q > 0 && (base & ~s.hold[e]) != 0u) {
+        const unsigned long long k =
+            ((unsigned long long)(unsigned)q << 32) | (0xffffffffu - unsigned(x));
+        ebest = k > ebest ? k : ebest;
+      }
+    }
+    ebest = warp_max_u64(ebest);
+    if (ebest == 0ull) {
+      if (lane == d) stuck = true;
+      continue;
+    }
+    const int e = d * Eh + int(0xffffffffu - unsigned(ebest & 0xffffffffu));
+    const int q = int(ebest >> 32);
+    const unsigned hold = s.hold[e];
+    const bool elig = ((base >> lane) & 1u) && !((hold >> lane) & 1u);
+    const bool cov = ((e / Eh) / gpn == lane / gpn) || ((hold & node_mask) != 0u);
+    const unsigned long long rkey =
+        elig ? (((unsigned long long)cov << 40) | ((unsigned long long)(unsigned)load << 5) |
+                unsigned(lane))
+             : ~0ull;
+    const unsigned long long rbest = warp_min_u64(rkey);
+    const int r = int(rbest & 31u);
+    const int rload = int((rbest >> 5) & 0x7fffffffull);
+    int m = dload - T;
+    m = min(m, T - rload);
+    m = min(m, q);
+    if (lane == r) {
+      s.repe[r * R + nfill] = e;
+      s.repq[r * R + nfill] = m;
+      ++nfill;
+      load += m;
+    }
+    if (lane == d) load -= m;
+    if (lane == 0) {
+      s.hq[e] = q - m;
+      s.hold[e] = hold | (1u << r);
+    }
+    __syncwarp();
+  }
+  if (lane < P) a.load_after[lane] = load;
+  int mx = lane < P ? load : 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(kFull, mx, o));
+  const int nrep = warp_sum(lane < P ? nfill : 0);
+  if (lane == 0) {
+    s.misc[kMiscMax] = mx;
+    s.misc[kMiscNrep] = nrep;
+    s.misc[kMiscIters] = iters;
+  }
+}
+
+__global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
+  extern __shared__ __align__(16) char smem_raw[];
+  PlannerSmem s = carve(smem_raw, a);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int P = a.P, E = a.E, R = a.R, Eh = a.Eh, G = Eh + R;
+
+  const int bad = a.flags[kFlagBadIds];
+  if (bad) {
+    if (tid == 0) {
+      a.stats[ZB_STAT_STATUS] = ZB_ERR_BAD_ID;
+      a.stats[ZB_STAT_BAD_IDS] = bad;
+      for (int k = 1; k < ZB_STATS_LEN; ++k)
+        if (k != ZB_STAT_BAD_IDS) a.stats[k] = 0;
+    }
+    return;
+  }
+
+  // T_e and the initial home quotas
+  for (int x = tid; x < P * E; x += kPlanThreads) s.cnt[x] = a.cnt[x];
+  __syncthreads();
+  for (int e = tid; e < E; e += kPlanThreads) {
+    int t = 0;
+    for (int i = 0; i < P; ++i) t += s.cnt[i * E + e];
+    s.hq[e] = t;
+    s.hold[e] = 0u;
+  }
+  for (int x = tid; x < P * R; x += kPlanThreads) {
+    s.repe[x] = -1;
+    s.repq[x] = 0;
+  }
+  if (tid == 0) s.misc[kMiscErr] = 0;
+  __syncthreads();
+
+  if (warp == 0) {
+    // L_j and the water level T = ceil(sum_r L_r / P)
+    int L = 0;
+    if (lane < P)
+      for (int e = lane * Eh; e < (lane + 1) * Eh; ++e) L += s.hq[e];
+    if (lane < P) a.load_before[lane] = L;
+    const long long total = warp_sum64(lane < P ? (long long)L : 0ll);
+    const int T = int((total + P - 1) / P);
+    if (lane == 0) s.misc[kMiscT] = T;
+    greedy_warp(a, s, T, lane);
+  }
+  __syncthreads();
+
+  const int T = s.misc[kMiscT];
+  const int max_load = s.misc[kMiscMax];
+  // plan tables
+  for (int e = tid; e < E; e += kPlanThreads) a.home_quota[e] = s.hq[e];
+  for (int x = tid; x < P * R; x += kPlanThreads) {
+    a.rep_expert[x] = s.repe[x];
+    a.rep_quota[x] = s.repq[x];
+  }
+  // hosts per expert and their first segment index (one warp scans E)
+  if (warp == 0) {
+    int carry = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      const int nh = e < E ? 1 + __popc(s.hold[e]) : 0;
+      const int inc = warp_incl_scan(nh, lane);
+      if (e < E) s.hoff[e] = carry + inc - nh;
+      carry += __shfl_sync(kFull, inc, 31);
+    }
+    if (lane == 0) s.hoff[E] = carry;
+  }
+  // cu_seqlens: exclusive prefix of each rank's group receipts (exact quotas)
+  for (int j = warp; j < P; j += kPlanWarps) {
+    int carry = 0;
+    int32_t* cu = s.cu + j * (G + 1);
+    if (lane == 0) cu[0] = 0;
+    for (int g0 = 0; g0 < G; g0 += 32) {
+      const int g = g0 + lane;
+      int v = 0;
+      if (g < G) v = g < Eh ? s.hq[j * Eh + g] : s.repq[j * R + (g - Eh)];
+      const int inc = warp_incl_scan(v, lane);
+      if (g < G) cu[g + 1] = carry + inc;
+      carry += __shfl_sync(kFull, inc, 31);
+    }
+  }
+  __syncthreads();
+  for (int x = tid; x < P * (G + 1); x += kPlanThreads) a.cu_seqlens[x] = s.cu[x];
+  for (int e = tid; e <= E; e += kPlanThreads) a.hoff[e] = s.hoff[e];
+
+  const bool capacity = max_load > a.cap;
+  long long cost_part = 0;
+  if (!capacity) {
+    // Transport of eq. (1), one warp per expert, lane = source rank.
+    int32_t* Mw = s.M + warp * 32 * 32;
+    int32_t* qw = s.q + warp * 32;
+    for (int e = warp; e < E; e += kPlanWarps) {
+      const int h0 = e / Eh;
+      const unsigned hostmask = s.hold[e] | (1u << h0);
+      const int nh = __popc(hostmask);
+      int dres = lane < P ? s.cnt[lane * E + e] : 0;
+      // host index of lane's own rank, its quota and group
+      const bool is_host = lane < P && ((hostmask >> lane) & 1u);
+      const int my_t = __popc(hostmask & ((1u << lane) - 1u));
+      for (int t = 0; t < nh; ++t) Mw[t * 32 + lane] = 0;
+      __syncwarp();
+      if (is_host) {
+        int q = 0;
+        if (lane == h0) {
+          q = s.hq[e];
+        } else {
+          for (int r = 0; r < R; ++r)
+            if (s.repe[lane * R + r] == e) q = s.repq[lane * R + r];
+        }
+        const int take = min(dres, q);  // phase 0: the host's own rank, a = 0
+        Mw[my_t * 32 + lane] = take;
+        dres -= take;
+        qw[my_t] = q - take;
+      }
+      __syncwarp();
+      const int nlev = a.gpn > 1 ? 2 : 1;
+      for (int l = 0; l < nlev; ++l) {
+        const int lev = l == 0 ? 1 : 4;
+        unsigned hm = hostmask;
+        for (int t = 0; t < nh; ++t) {
+          const int j = __ffs(hm) - 1;
+          hm &= hm - 1u;
+          const int rem = qw[t];
+          const bool el = lane < P && cost_a(lane, j, a.gpn) == lev;
+          const int v = el ? dres : 0;
+          const int inc = warp_incl_scan(v, lane);
+          const int take = max(0, min(v, rem - (inc - v)));
+          const int tot = warp_sum(take);
+          Mw[t * 32 + lane] += take;
+          dres -= take;
+          __syncwarp();
+          if (lane == 0) qw[t] = rem - tot;
+          __syncwarp();
+        }
+      }
+      if (warp_sum(dres != 0) != 0 && lane == 0) atomicExch(&s.misc[kMiscErr], 1);
+      // locality cost, segment starts and the segment table of each source
+      {
+        unsigned hm = hostmask;
+        for (int t = 0; t < nh; ++t) {
+          const int j = __ffs(hm) - 1;
+          hm &= hm - 1u;
+          const int m = Mw[t * 32 + lane];
+          cost_part += (long long)cost_a(lane, j, a.gpn) * m;
+          const int inc = warp_incl_scan(m, lane);
+          __syncwarp();
+          Mw[t * 32 + lane] = inc;  // inclusive prefix over sources
+        }
+        __syncwarp();
+      }
+      if (lane < P) {
+        int2* seg = a.seg + int64_t(lane) * a.seg_width + s.hoff[e];
+        int idx = 0, cum = 0;
+        for (int lv = 0; lv < 3; ++lv) {
+          const int want = lv == 0 ? 0 : (lv == 1 ? 1 : 4);
+          unsigned hm = hostmask;
+          for (int t = 0; t < nh; ++t) {
+            const int j = __ffs(hm) - 1;
+            hm &= hm - 1u;
+            if (cost_a(lane, j, a.gpn) != want) continue;
+            const int inc = Mw[t * 32 + lane];
+            const int prev = lane > 0 ? Mw[t * 32 + lane - 1] : 0;
+            int grp;
+            if (j == h0) {
+              grp = e - h0 * Eh;
+            } else {
+              grp = Eh;
+              for (int r = 0; r < R; ++r)
+                if (s.repe[j * R + r] == e) grp = Eh + r;
+            }
+            cum += inc - prev;
+            const int base = j * a.cap + s.cu[j * (G + 1) + grp] + prev;
+            seg[idx++] = make_int2(cum, base);
+          }
+        }
+      }
+      __syncwarp();
+    }
+  }
+  cost_part = warp_sum64(cost_part);
+  __shared__ unsigned long long s_cost;
+  if (tid == 0) s_cost = 0ull;
+  __syncthreads();
+  if (lane == 0) atomicAdd(&s_cost, (unsigned long long)cost_part);
+  __syncthreads();
+  if (tid == 0) {
+    int status = ZB_OK;
+    if (capacity)
+      status = ZB_ERR_CAPACITY;
+    else if (s.misc[kMiscErr])
+      status = ZB_ERR_INVALID;  // unreachable: transport always closes
+    else if (max_load > T)
+      status = ZB_WARN_UNBALANCED;
+    a.stats[ZB_STAT_STATUS] = status;
+    a.stats[ZB_STAT_MAX_LOAD] = max_load;
+    a.stats[ZB_STAT_N_REPLICAS] = s.misc[kMiscNrep];
+    a.stats[ZB_STAT_N_ITERS] = s.misc[kMiscIters];
+    a.stats[ZB_STAT_WATER_LEVEL] = T;
+    a.stats[ZB_STAT_LOCALITY_COST] = capacity ? 0 : (long long)s_cost;
+    a.stats[ZB_STAT_BAD_IDS] = 0;
+    a.stats[7] = 0;
+  }
+}
+
+// ------------------------------------------------------------------ step 3
+
+constexpr int kAssignWarps = kChunkThreads / 32;
+constexpr int kPerWarp = kChunk / kAssignWarps;  // 256 entries, 8 steps of 32
+
+__global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
+  if (a.stats[ZB_STAT_STATUS] < 0) return;  // bad ids or capacity: no rows
+  __shared__ int32_t wh[kAssignWarps][kMaxE];  // per-warp running position
+  const int c = blockIdx.x, i = blockIdx.y, tid = threadIdx.x, lane = tid & 31,
+            warp = tid >> 5;
+  const int E = a.E;
+  const int64_t nk = int64_t(a.S) * a.K;
+  const int64_t start = int64_t(c) * kChunk;
+  const int n = (nk - start) < kChunk ? int(nk - start) : kChunk;
+  const int32_t* src = a.ids + int64_t(i) * nk + start;
+
+  // pass 1: per-warp histogram of the warp's slice
+  for (int x = tid; x < kAssignWarps * kMaxE; x += kChunkThreads) (&wh[0][0])[x] = 0;
+  __syncthreads();
+  const int w0 = warp * kPerWarp;
+  for (int t0 = 0; t0 < kPerWarp; t0 += 32) {
+    const int t = w0 + t0 + lane;
+    const int e = t < n ? __ldg(src + t) : -1;
+    const unsigned peers = __match_any_sync(kFull, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) wh[warp][e] += __popc(peers);
+  }
+  __syncthreads();
+  // exclusive prefix: earlier chunks of this source, then earlier warps
+  for (int e = tid; e < E; e += kChunkThreads) {
+    int run = 0;
+    const int32_t* ch = a.chunk_hist + int64_t(i) * a.nchunk * E + e;
+    for (int cc = 0; cc < c; ++cc) run += ch[int64_t(cc) * E];
+    for (int w = 0; w < kAssignWarps; ++w) {
+      const int v = wh[w][e];
+      wh[w][e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  // pass 2: stable position of each entry, then its segment and row
+  const int2* segrow = a.seg + int64_t(i) * a.seg_width;
+  for (int t0 = 0; t0 < kPerWarp; t0 += 32) {
+    const int t = w0 + t0 + lane;
+    const int e = t < n ? __ldg(src + t) : -1;
+    const unsigned peers = __match_any_sync(kFull, e);
+    int p = 0;
+    if (e >= 0) p = wh[warp][e] + __popc(peers & ((1u << lane) - 1u));
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(peers) - 1) wh[warp][e] += __popc(peers);
+    __syncwarp();
+    if (e >= 0) {
+      const int h_begin = a.hoff[e], h_end = a.hoff[e + 1];
+      int prev = 0, row = -1;
+      for (int h = h_begin; h < h_end; ++h) {
+        const int2 sg = segrow[h];
+        if (p < sg.x) {
+          row = sg.y + (p - prev);
+          break;
+        }
+        prev = sg.x;
+      }
+      const int64_t g = int64_t(i) * nk + start + t;
+      a.dst_row[g] = row;
+      if (a.row_src && row >= 0 && int64_t(row) < int64_t(a.P) * a.cap)
+        a.row_src[row] = int32_t(g);
+    }
+  }
+}
+
+}  // namespace
+
+size_t planner_smem_bytes(const zb_config& c) {
+  const int Eh = c.E / c.P;
+  size_t words = size_t(c.P) * c.E + 2 * size_t(c.E) + 2 * size_t(c.P) * c.R +
+                 size_t(c.P) * (Eh + c.R + 1) + size_t(c.E + 1) + kPlanWarps * 32 + 16;
+  words = (words + 3) & ~size_t(3);
+  words += size_t(kPlanWarps) * 32 * 32;
+  return words * sizeof(int32_t);
+}
+
+cudaError_t launch_hist(const PlanArgs& a, cudaStream_t s) {
+  if (a.nchunk == 0) return cudaSuccess;
+  k_hist<<<dim3(a.nchunk, a.P), kChunkThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_planner(const PlanArgs& a, size_t smem, cudaStream_t s) {
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    err = cudaFuncSetAttribute(k_planner, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               200 * 1024);
+    if (err != cudaSuccess) return err;
+    configured[dev] = true;
+  }
+  k_planner<<<1, kPlanThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_assign(const PlanArgs& a, cudaStream_t s) {
+  if (a.nchunk == 0) return cudaSuccess;
+  k_assign<<<dim3(a.nchunk, a.P), kChunkThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace zb

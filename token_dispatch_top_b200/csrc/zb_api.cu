@@ -1,0 +1,138 @@
+// zb_api.cu -- the C ABI declared in include/zb.h: validation, workspace
+// sizing, status codes and the launch sequence of each call.  No allocation
+// and no synchronisation happen here, except the documented stream
+// synchronisation of zb_plan_status.
+#include <cstring>
+
+#include "zb_internal.cuh"
+
+using zb::Workspace;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int plan_buffers_ok(const zb_config& c, const zb_plan_t* p) {
+  if (!p) return 0;
+  if (!p->cnt || !p->home_quota || !p->load_before || !p->load_after || !p->cu_seqlens ||
+      !p->stats)
+    return 0;
+  if (c.R > 0 && (!p->rep_expert || !p->rep_quota)) return 0;
+  if (c.S > 0 && !p->dst_row) return 0;
+  return 1;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* zb_strerror(int status) {
+  switch (status) {
+    case ZB_OK: return "ok";
+    case ZB_WARN_UNBALANCED: return "unbalanced: the replica slots do not permit the water level";
+    case ZB_ERR_INVALID: return "invalid configuration, pointer, size or alignment";
+    case ZB_ERR_CAPACITY: return "planned rank load exceeds cap_rows";
+    case ZB_ERR_BAD_ID: return "routing id outside [0, E)";
+    case ZB_ERR_TIMEOUT: return "a bounded device wait gave up";
+    case ZB_ERR_CUDA: return "CUDA runtime error";
+    default: return "unknown status";
+  }
+}
+
+int zb_validate(const zb_config* c) {
+  if (!c) return ZB_ERR_INVALID;
+  if (c->P < 1 || c->P > zb::kMaxP) return ZB_ERR_INVALID;
+  if (c->E < c->P || c->E > zb::kMaxE || c->E % c->P != 0) return ZB_ERR_INVALID;
+  if (c->K < 1 || c->K > 16) return ZB_ERR_INVALID;
+  if (c->S < 0) return ZB_ERR_INVALID;
+  if (c->H < 8 || c->H % 8 != 0) return ZB_ERR_INVALID;
+  if (c->R < 0 || c->R > c->P - 1) return ZB_ERR_INVALID;
+  if (!(c->C >= 0.0f && c->C < 1.0f)) return ZB_ERR_INVALID;
+  if (c->gpus_per_node < 1 || c->P % c->gpus_per_node != 0) return ZB_ERR_INVALID;
+  const int64_t sk = int64_t(c->S) * c->K;
+  if (sk > INT32_MAX) return ZB_ERR_INVALID;
+  if (int64_t(c->cap_rows) < sk) return ZB_ERR_INVALID;
+  if (int64_t(c->P) * sk > INT32_MAX) return ZB_ERR_INVALID;
+  if (int64_t(c->P) * c->cap_rows > INT32_MAX) return ZB_ERR_INVALID;
+  return ZB_OK;
+}
+
+size_t zb_workspace_bytes(const zb_config* c) {
+  if (zb_validate(c) != ZB_OK) return 0;
+  return zb::workspace_layout(*c).bytes;
+}
+
+int zb_plan(const zb_config* c, const int32_t* ids, const zb_plan_t* plan, void* ws,
+            size_t ws_bytes, void* stream) {
+  if (zb_validate(c) != ZB_OK) return ZB_ERR_INVALID;
+  if (!plan_buffers_ok(*c, plan)) return ZB_ERR_INVALID;
+  const Workspace w = zb::workspace_layout(*c);
+  if (!ws || ws_bytes < w.bytes || (reinterpret_cast<uintptr_t>(ws) & 255u)) return ZB_ERR_INVALID;
+  if (c->S > 0 && !ids) return ZB_ERR_INVALID;
+  cudaStream_t s = as_stream(stream);
+  char* base = static_cast<char*>(ws);
+
+  zb::PlanArgs a{};
+  a.P = c->P; a.E = c->E; a.K = c->K; a.S = c->S; a.R = c->R; a.Eh = c->E / c->P;
+  a.gpn = c->gpus_per_node; a.cap = c->cap_rows;
+  a.nchunk = w.nchunk; a.seg_width = w.seg_width;
+  a.ids = ids;
+  a.cnt = plan->cnt; a.rep_expert = plan->rep_expert; a.rep_quota = plan->rep_quota;
+  a.home_quota = plan->home_quota; a.load_before = plan->load_before;
+  a.load_after = plan->load_after; a.cu_seqlens = plan->cu_seqlens; a.dst_row = plan->dst_row;
+  a.row_src = plan->row_src; a.stats = plan->stats;
+  a.flags = reinterpret_cast<int32_t*>(base + w.off_flags);
+  a.chunk_hist = reinterpret_cast<int32_t*>(base + w.off_chunk_hist);
+  a.hoff = reinterpret_cast<int32_t*>(base + w.off_hoff);
+  a.seg = reinterpret_cast<int2*>(base + w.off_seg);
+
+  if (cudaMemsetAsync(a.flags, 0, sizeof(int32_t) * zb::kFlagWords, s) != cudaSuccess)
+    return ZB_ERR_CUDA;
+  if (cudaMemsetAsync(a.cnt, 0, sizeof(int32_t) * size_t(c->P) * c->E, s) != cudaSuccess)
+    return ZB_ERR_CUDA;
+  if (a.row_src &&
+      cudaMemsetAsync(a.row_src, 0xff, sizeof(int32_t) * size_t(c->P) * c->cap_rows, s) !=
+          cudaSuccess)
+    return ZB_ERR_CUDA;
+  if (zb::launch_hist(a, s) != cudaSuccess) return ZB_ERR_CUDA;
+  if (zb::launch_planner(a, zb::planner_smem_bytes(*c), s) != cudaSuccess) return ZB_ERR_CUDA;
+  if (zb::launch_assign(a, s) != cudaSuccess) return ZB_ERR_CUDA;
+  return ZB_OK;
+}
+
+int zb_plan_status(const zb_config* c, const zb_plan_t* plan, void* stream, int32_t* max_load) {
+  if (zb_validate(c) != ZB_OK || !plan || !plan->stats) return ZB_ERR_INVALID;
+  int64_t st[ZB_STATS_LEN];
+  cudaStream_t s = as_stream(stream);
+  if (cudaMemcpyAsync(st, plan->stats, sizeof(st), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return ZB_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ZB_ERR_CUDA;
+  if (max_load) *max_load = int32_t(st[ZB_STAT_MAX_LOAD]);
+  return int(st[ZB_STAT_STATUS]);
+}
+
+int zb_dispatch(const zb_config* c, const zb_plan_t* plan, const uint16_t* hidden,
+                uint16_t* buf, void* stream) {
+  if (zb_validate(c) != ZB_OK || !plan || !plan->stats) return ZB_ERR_INVALID;
+  if (c->S > 0 && (!plan->dst_row || !hidden || !buf)) return ZB_ERR_INVALID;
+  if ((hidden && !aligned16(hidden)) || (buf && !aligned16(buf))) return ZB_ERR_INVALID;
+  if (zb::launch_dispatch(c->P, c->S, c->K, c->H, c->cap_rows, plan->dst_row, plan->stats,
+                          hidden, buf, as_stream(stream)) != cudaSuccess)
+    return ZB_ERR_CUDA;
+  return ZB_OK;
+}
+
+int zb_combine(const zb_config* c, const zb_plan_t* plan, const uint16_t* y, const float* w,
+               uint16_t* out, void* stream) {
+  if (zb_validate(c) != ZB_OK || !plan || !plan->stats) return ZB_ERR_INVALID;
+  if (c->S > 0 && (!plan->dst_row || !y || !w || !out)) return ZB_ERR_INVALID;
+  if ((y && !aligned16(y)) || (out && !aligned16(out))) return ZB_ERR_INVALID;
+  if (zb::launch_combine(c->P, c->S, c->K, c->H, c->cap_rows, plan->dst_row, plan->stats, y, w,
+                         out, as_stream(stream)) != cudaSuccess)
+    return ZB_ERR_CUDA;
+  return ZB_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,93 @@
+// zb_internal.cuh -- definitions shared by the device library's translation
+// units: workspace layout, launch constants and the kernel declarations.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "zb.h"
+
+namespace zb {
+
+// Entries of one source rank handled by one CTA of the histogram and the
+// assignment kernels.
+constexpr int kChunk = 2048;
+constexpr int kChunkThreads = 256;
+constexpr int kMaxE = 384;
+constexpr int kMaxP = 32;
+constexpr int kPlanThreads = 512;  // 16 warps
+constexpr int kPlanWarps = kPlanThreads / 32;
+
+// Workspace flag words.
+enum { kFlagBadIds = 0, kFlagInternal = 1, kFlagWords = 64 };
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Layout of the scratch workspace (all offsets 256-byte aligned):
+//   flags      int32 [kFlagWords]
+//   chunk_hist int32 [P][nchunk][E]    per-chunk expert counts
+//   hoff       int32 [E+1]             first segment of expert e in a row of seg
+//   seg        int2  [P][E + P*R]      per (source i, expert e): the hosts in
+//                                      the order source i fills them, as
+//                                      (cumulative end count, base row)
+struct Workspace {
+  int nchunk;
+  int seg_width;
+  size_t off_flags, off_chunk_hist, off_hoff, off_seg, bytes;
+};
+
+inline Workspace workspace_layout(const zb_config& c) {
+  Workspace w{};
+  const int64_t nk = int64_t(c.S) * c.K;
+  w.nchunk = int(ceil_div(nk, kChunk));
+  w.seg_width = c.E + c.P * c.R;
+  size_t o = 0;
+  w.off_flags = o;
+  o = align256(o + sizeof(int32_t) * kFlagWords);
+  w.off_chunk_hist = o;
+  o = align256(o + sizeof(int32_t) * size_t(c.P) * w.nchunk * c.E);
+  w.off_hoff = o;
+  o = align256(o + sizeof(int32_t) * size_t(c.E + 1));
+  w.off_seg = o;
+  o = align256(o + sizeof(int2) * size_t(c.P) * w.seg_width);
+  w.bytes = o;
+  return w;
+}
+
+// Kernel parameter block shared by the plan kernels.
+struct PlanArgs {
+  int P, E, K, S, R, Eh, gpn, cap;
+  int nchunk, seg_width;
+  const int32_t* ids;
+  int32_t* cnt;
+  int32_t* rep_expert;
+  int32_t* rep_quota;
+  int32_t* home_quota;
+  int32_t* load_before;
+  int32_t* load_after;
+  int32_t* cu_seqlens;
+  int32_t* dst_row;
+  int32_t* row_src;
+  int64_t* stats;
+  int32_t* flags;
+  int32_t* chunk_hist;
+  int32_t* hoff;
+  int2* seg;
+};
+
+size_t planner_smem_bytes(const zb_config& c);
+
+cudaError_t launch_hist(const PlanArgs& a, cudaStream_t s);
+cudaError_t launch_planner(const PlanArgs& a, size_t smem, cudaStream_t s);
+cudaError_t launch_assign(const PlanArgs& a, cudaStream_t s);
+
+cudaError_t launch_dispatch(int P, int S, int K, int H, int cap, const int32_t* dst_row,
+                            const int64_t* stats, const uint16_t* hidden, uint16_t* buf,
+                            cudaStream_t s);
+cudaError_t launch_combine(int P, int S, int K, int H, int cap, const int32_t* dst_row,
+                           const int64_t* stats, const uint16_t* y, const float* w,
+                           uint16_t* out, cudaStream_t s);
+
+}  // namespace zb

@@ -1,0 +1,203 @@
+"""Python binding of libzb (ctypes): argument marshalling only.
+
+Every step of plan, dispatch and combine runs in the CUDA kernels of
+``libzb.so``; this module passes ``torch.Tensor`` device pointers, sizes and
+the current CUDA stream to the C ABI declared in ``include/zb.h``.  There is
+no CPU fallback: if the library is missing or fails to load, every call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libzb.so")
+
+OK = 0
+WARN_UNBALANCED = 1
+ERR_INVALID = -1
+ERR_CAPACITY = -2
+ERR_BAD_ID = -3
+ERR_TIMEOUT = -4
+ERR_CUDA = -5
+
+STAT_STATUS, STAT_MAX_LOAD, STAT_N_REPLICAS, STAT_N_ITERS, STAT_WATER_LEVEL, \
+    STAT_LOCALITY_COST, STAT_BAD_IDS = range(7)
+STATS_LEN = 8
+
+EXPORTS = ("zb_strerror", "zb_validate", "zb_workspace_bytes", "zb_plan", "zb_plan_status",
+           "zb_dispatch", "zb_combine")
+
+
+class ZbError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {strerror(status)} (status {status})")
+        self.status = status
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [("P", ctypes.c_int), ("E", ctypes.c_int), ("K", ctypes.c_int),
+                ("S", ctypes.c_int), ("H", ctypes.c_int), ("R", ctypes.c_int),
+                ("C", ctypes.c_float), ("gpus_per_node", ctypes.c_int),
+                ("cap_rows", ctypes.c_int)]
+
+
+class _Plan(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("cnt", "rep_expert", "rep_quota", "home_quota", "load_before", "load_after",
+                 "cu_seqlens", "dst_row", "row_src", "stats")]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libzb.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libzb.so not built at {LIB_PATH}; run "
+                              "`python -m token_dispatch_top_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, cfgp, planp = ctypes.c_void_p, ctypes.POINTER(_Cfg), ctypes.POINTER(_Plan)
+        lib.zb_strerror.argtypes = [ctypes.c_int]
+        lib.zb_strerror.restype = ctypes.c_char_p
+        lib.zb_validate.argtypes = [cfgp]
+        lib.zb_workspace_bytes.argtypes = [cfgp]
+        lib.zb_workspace_bytes.restype = ctypes.c_size_t
+        lib.zb_plan.argtypes = [cfgp, vp, planp, vp, ctypes.c_size_t, vp]
+        lib.zb_plan_status.argtypes = [cfgp, planp, vp, ctypes.POINTER(ctypes.c_int32)]
+        lib.zb_dispatch.argtypes = [cfgp, planp, vp, vp, vp]
+        lib.zb_combine.argtypes = [cfgp, planp, vp, vp, vp, vp]
+        _lib = lib
+    return _lib
+
+
+def strerror(status: int) -> str:
+    return load().zb_strerror(int(status)).decode()
+
+
+@dataclass(frozen=True)
+class Config:
+    """Problem shape; see ``zb_config`` in include/zb.h for the bounds."""
+    P: int
+    E: int
+    K: int
+    S: int
+    H: int
+    R: int
+    C: float = 0.0
+    gpus_per_node: int = 1
+    cap_rows: int | None = None  # default S*K
+
+    @property
+    def cap(self) -> int:
+        return self.S * self.K if self.cap_rows is None else self.cap_rows
+
+    @property
+    def Eh(self) -> int:
+        return self.E // self.P
+
+    def c(self) -> _Cfg:
+        return _Cfg(self.P, self.E, self.K, self.S, self.H, self.R, float(self.C),
+                    self.gpus_per_node, self.cap)
+
+
+def validate(cfg: Config) -> int:
+    return int(load().zb_validate(ctypes.byref(cfg.c())))
+
+
+def workspace_bytes(cfg: Config) -> int:
+    return int(load().zb_workspace_bytes(ctypes.byref(cfg.c())))
+
+
+class Plan:
+    """Device buffers of one plan plus its scratch workspace (torch-owned)."""
+
+    def __init__(self, cfg: Config, device, with_row_src: bool = True):
+        if validate(cfg) != OK:
+            raise ZbError(ERR_INVALID, f"config {cfg}")
+        i32 = dict(dtype=torch.int32, device=device)
+        P, E, R = cfg.P, cfg.E, cfg.R
+        self.cfg = cfg
+        self.cnt = torch.empty((P, E), **i32)
+        self.rep_expert = torch.empty((P, R), **i32)
+        self.rep_quota = torch.empty((P, R), **i32)
+        self.home_quota = torch.empty((E,), **i32)
+        self.load_before = torch.empty((P,), **i32)
+        self.load_after = torch.empty((P,), **i32)
+        self.cu_seqlens = torch.empty((P, cfg.Eh + R + 1), **i32)
+        self.dst_row = torch.empty((P, cfg.S, cfg.K), **i32)
+        self.row_src = torch.empty((P, cfg.cap), **i32) if with_row_src else None
+        self.stats = torch.zeros((STATS_LEN,), dtype=torch.int64, device=device)
+        self.ws_bytes = workspace_bytes(cfg)
+        self.workspace = torch.empty((self.ws_bytes + 256,), dtype=torch.uint8, device=device)
+        self.ws_ptr = (self.workspace.data_ptr() + 255) & ~255  # 256-byte aligned
+        self._c = cfg.c()
+
+        def p(t):
+            return None if t is None or t.numel() == 0 else t.data_ptr()
+        self._p = _Plan(p(self.cnt), p(self.rep_expert), p(self.rep_quota), p(self.home_quota),
+                        p(self.load_before), p(self.load_after), p(self.cu_seqlens),
+                        p(self.dst_row), p(self.row_src), p(self.stats))
+
+
+def _stream(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _check(t: torch.Tensor, shape, dtype, name):
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous() \
+            or not t.is_cuda:
+        raise ZbError(ERR_INVALID, f"{name}: want contiguous cuda {dtype} {tuple(shape)}, got "
+                                   f"{t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def plan(p: Plan, topk_ids: torch.Tensor, stream=None) -> None:
+    """Steps 1-3 (asynchronous).  ``topk_ids``: int32 [P,S,K] on the device."""
+    cfg = p.cfg
+    _check(topk_ids, (cfg.P, cfg.S, cfg.K), torch.int32, "topk_ids")
+    st = load().zb_plan(ctypes.byref(p._c), topk_ids.data_ptr(), ctypes.byref(p._p),
+                        p.ws_ptr, p.ws_bytes, _stream(stream))
+    if st != OK:
+        raise ZbError(st, "zb_plan")
+
+
+def plan_status(p: Plan, stream=None) -> tuple[int, int]:
+    """Synchronise the stream and return (status, max_load) of the plan."""
+    ml = ctypes.c_int32(0)
+    st = load().zb_plan_status(ctypes.byref(p._c), ctypes.byref(p._p), _stream(stream),
+                               ctypes.byref(ml))
+    if st in (ERR_INVALID, ERR_CUDA):
+        raise ZbError(st, "zb_plan_status")
+    return int(st), int(ml.value)
+
+
+def dispatch(p: Plan, hidden: torch.Tensor, buf: torch.Tensor, stream=None) -> None:
+    """Step 4 (asynchronous): ``hidden`` bf16 [P,S,H] -> ``buf`` bf16 [P,cap,H]."""
+    cfg = p.cfg
+    _check(hidden, (cfg.P, cfg.S, cfg.H), torch.bfloat16, "hidden")
+    _check(buf, (cfg.P, cfg.cap, cfg.H), torch.bfloat16, "buf")
+    st = load().zb_dispatch(ctypes.byref(p._c), ctypes.byref(p._p), hidden.data_ptr(),
+                            buf.data_ptr(), _stream(stream))
+    if st != OK:
+        raise ZbError(st, "zb_dispatch")
+
+
+def combine(p: Plan, y: torch.Tensor, topk_weights: torch.Tensor, out: torch.Tensor,
+            stream=None) -> None:
+    """Step 5 (asynchronous): ``y`` bf16 [P,cap,H], ``topk_weights`` fp32 [P,S,K]
+    -> ``out`` bf16 [P,S,H]."""
+    cfg = p.cfg
+    _check(y, (cfg.P, cfg.cap, cfg.H), torch.bfloat16, "y")
+    _check(topk_weights, (cfg.P, cfg.S, cfg.K), torch.float32, "topk_weights")
+    _check(out, (cfg.P, cfg.S, cfg.H), torch.bfloat16, "out")
+    st = load().zb_combine(ctypes.byref(p._c), ctypes.byref(p._p), y.data_ptr(),
+                           topk_weights.data_ptr(), out.data_ptr(), _stream(stream))
+    if st != OK:
+        raise ZbError(st, "zb_combine")
