@@ -10,8 +10,9 @@ to the combine are the dispatched rows themselves (identity experts), so the
 step moves exactly the dispatch and combine traffic.
 
 * ``value``: tokens/s over all ranks, device-timed with CUDA events with the
-  inputs resident in HBM; L2 (126 MB) is flushed by a 256 MB write before
-  every step, outside the timed events.
+  inputs resident in HBM; L2 (126 MB) is flushed before every step, outside
+  the timed events, by a 256 MB write followed by a 256 MB read (so no dirty
+  flush lines are written back inside the timed step).
 * ``e2e``: the same metric through the public API with pinned host buffers:
   each step copies ids, weights and hidden rows host->device, runs the path,
   and copies the combined rows and the plan status back.
@@ -76,9 +77,9 @@ def read_peaks() -> tuple[float, str]:
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(files) -> str:
     h = hashlib.sha256()
-    for name in ("move_kernels.cu", "plan_kernels.cu", "zb_internal.cuh"):
+    for name in files:
         with open(os.path.join(ROOT, "token_dispatch_top_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -93,7 +94,7 @@ def recorded_traffic(kernel: str) -> float | None:
             rec = json.load(f)
     except (OSError, ValueError):
         return None
-    if rec.get("source_hash") != kernel_source_hash():
+    if rec.get("source_hash") != kernel_source_hash(rec.get("source_files", [])):
         return None
     v = rec.get("kernels", {}).get(kernel, {}).get("dram_bytes_per_launch")
     return float(v) if v is not None else None
@@ -154,6 +155,22 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
                 "samples": len(rows)}
+
+
+def max_over_ranks(values, dist, device):
+    """Element-wise max of per-rank timings (the slowest rank sets the time)."""
+    if dist is None:
+        return list(values)
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def weak_scaling_value(tokens_per_rank: int, world: int, total_ms: float, steps: int) -> float:
+    """Tokens/s of the whole job: every rank processes its own batch per step,
+    and the job takes the slowest rank's time."""
+    return tokens_per_rank * world / (total_ms / steps / 1000.0)
 
 
 def oracle_steps(wl, ids, w, hidden_bits, budget_s: float, min_steps: int = 1):
@@ -257,6 +274,15 @@ def run_ours(args, wl, rank, world, local_rank):
     buf = torch.empty((P, cap, H), dtype=torch.bfloat16, device=dev)
     out = torch.empty((P, S, H), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush_src = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        # write a buffer twice the size of L2, then read another one, so the
+        # step starts with L2 holding only clean lines of no use to it
+        flush.zero_()
+        torch.sum(flush_src, out=flush_sink)
+
     stream = torch.cuda.current_stream()
 
     def step():
@@ -276,7 +302,7 @@ def run_ours(args, wl, rank, world, local_rank):
             dist.barrier()
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush_l2()
         step()
     barrier()
     n_ev = args.steps
@@ -285,7 +311,7 @@ def run_ours(args, wl, rank, world, local_rank):
         barrier()
         t0 = time.perf_counter()
         for k in range(args.steps):
-            flush.zero_()
+            flush_l2()
             ev[k][0].record(stream)
             zb.plan(plan, ids)
             ev[k][1].record(stream)
@@ -330,7 +356,7 @@ def run_ours(args, wl, rank, world, local_rank):
     e1 = torch.cuda.Event(enable_timing=True)
     e2e_ms = 0.0
     for _ in range(args.steps):
-        flush.zero_()
+        flush_l2()
         e0.record(stream)
         e2e_step()
         e1.record(stream)
@@ -343,19 +369,14 @@ def run_ours(args, wl, rank, world, local_rank):
     d2h = P * S * H * 2 + zb.STATS_LEN * 8
 
     # ---- max over ranks
-    vals = [step_ms, e2e_ms, sum(t_disp), sum(t_comb), sum(t_plan)]
-    if dist is not None:
-        tt = torch.tensor(vals, dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        vals = tt.tolist()
-    step_ms, e2e_ms, disp_ms, comb_ms, plan_ms = vals
+    step_ms, e2e_ms, disp_ms, comb_ms, plan_ms = max_over_ranks(
+        [step_ms, e2e_ms, sum(t_disp), sum(t_comb), sum(t_plan)], dist, dev)
     if rank != 0:
         return
 
-    tokens = wl.tokens * world
     ms_per_step = step_ms / args.steps
-    value = tokens / (ms_per_step / 1000.0)
-    e2e_value = tokens / (e2e_ms / args.steps / 1000.0)
+    value = weak_scaling_value(wl.tokens, world, step_ms, args.steps)
+    e2e_value = weak_scaling_value(wl.tokens, world, e2e_ms, args.steps)
     ab = algorithmic_bytes(wl)
     disp_ms_avg = disp_ms / args.steps
     comb_ms_avg = comb_ms / args.steps
@@ -379,7 +400,7 @@ def run_ours(args, wl, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": workload_desc(wl), "tokens_per_step_per_gpu": wl.tokens,
                    "accumulate": "f32", "experts": "identity (y = dispatched rows)",
-                   "l2": "flushed before every step by a 256 MB write (outside the timing)",
+                   "l2": "flushed before every step (outside the timing): a 256 MB write, then a 256 MB read",
                    "parallelism": f"replicas x{world}"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
