@@ -168,6 +168,35 @@ ZB_API int zb_plan(const zb_config *cfg, const int32_t *topk_ids, const zb_plan_
 ZB_API int zb_plan_status(const zb_config *cfg, const zb_plan_t *plan, void *stream,
                    int32_t *max_load);
 
+/* Size of the scratch array behind zb_plan_noalloc: 4 MiB.  A config is
+ * accepted there only if zb_workspace_bytes(cfg) <= this. */
+#define ZB_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/* zb_plan without a caller-provided workspace, for callers that cannot
+ * allocate device memory: for example a plugin enqueued by a host framework
+ * that owns every allocation and offers it no scratch buffer, or a serving
+ * loop that bans cudaMalloc/cudaFree on its hot path because they can
+ * synchronise the device.  The pages have no counterpart; this is a
+ * convenience of the library.
+ *
+ * Same arguments, results and errors as zb_plan, minus the workspace: the
+ * scratch is a fixed 4 MiB device array inside libzb that every GPU loading
+ * the library keeps until the process exits.  It allocates nothing and calls
+ * no allocating routine.
+ *  - Limit: returns ZB_ERR_INVALID, enqueueing nothing, when
+ *    zb_workspace_bytes(cfg) > ZB_NOALLOC_SCRATCH_BYTES (besides every reason
+ *    zb_plan gives).
+ *  - The scratch belongs to the calling thread's current device, so `stream`
+ *    must belong to that device too.  The first call on a device looks up the
+ *    array's device address (once per device) and caches it; make that first
+ *    call before any stream capture starts.
+ *  - Every call on a device shares the one array, which keeps what the last
+ *    call left in it; each call clears what it needs zeroed.  Calls whose work
+ *    overlaps on the GPU (two streams, or two host threads) race on the
+ *    array: order them on one stream or serialise them. */
+ZB_API int zb_plan_noalloc(const zb_config *cfg, const int32_t *topk_ids, const zb_plan_t *plan,
+                           void *stream);
+
 /* Step 4: buf[dst_row[i,s,k]][:] = hidden[i,s][:], bit for bit: each token row
  * is written into the fixed-shape, expert-grouped receive buffer of every rank
  * that serves one of its K experts (MoonEP, section on what it enforces: rows
