@@ -1,10 +1,13 @@
 // plan_kernels.cu -- steps 1-3 of an invocation on one GPU:
 //   k_hist     per-(source rank, chunk) expert histogram in shared memory
-//   k_planner  one CTA: water level, greedy replica placement (one warp, lanes
-//              = ranks), quotas, cu_seqlens, locality-first transport and the
-//              per-(source, expert) segment table
+//   k_planner  one CTA: route counts, water level, greedy replica placement
+//              (one warp, lanes = ranks), quotas, cu_seqlens, locality-first
+//              transport and the per-(source, expert) segment table
 //   k_assign   per-(source rank, chunk): stable rank of every entry among the
 //              source's entries of the same expert, then its destination row
+//
+// No kernel waits on another CTA: the chunk prefix each assignment CTA needs
+// is summed directly from the per-chunk histograms.
 //
 // Sources: ISER-MoE "Methodology / HALO-Q Scheduler" (Objective 1 water level,
 // stages 1, 2, 3, 5); Zepp "4.1 Expert Placement and Token Routing" (R slots
@@ -16,38 +19,32 @@ namespace zb {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
+constexpr int kPerThread = kChunk / kChunkThreads;  // entries per thread
 
-__device__ __forceinline__ int warp_sum(int v) {
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(kFull, v, o);
+    if (lane >= o) v += u;
+  }
   return v;
 }
+
 __device__ __forceinline__ long long warp_sum64(long long v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
   return v;
 }
-__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+
+// Sum of col[0], col[stride], ..., col[(n-1)*stride], eight loads in flight.
+__device__ __forceinline__ int strided_sum(const int32_t* col, int n, int64_t stride) {
+  int v = 0;
+  for (int c = 0; c < n; c += 8) {
+    int x[8];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    unsigned long long u = __shfl_xor_sync(kFull, v, o);
-    v = u > v ? u : v;
-  }
-  return v;
-}
-__device__ __forceinline__ unsigned long long warp_min_u64(unsigned long long v) {
+    for (int u = 0; u < 8; ++u) x[u] = c + u < n ? col[int64_t(c + u) * stride] : 0;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    unsigned long long u = __shfl_xor_sync(kFull, v, o);
-    v = u < v ? u : v;
-  }
-  return v;
-}
-__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int u = __shfl_up_sync(kFull, v, o);
-    if (lane >= o) v += u;
+    for (int u = 0; u < 8; ++u) v += x[u];
   }
   return v;
 }
@@ -61,34 +58,40 @@ __device__ __forceinline__ int cost_a(int i, int j, int gpn) {
 
 // ------------------------------------------------------------------ step 1
 
+// One CTA per (chunk c, source rank i).  Thread t handles entries
+// t + kChunkThreads*u, u < kPerThread, all loaded before the first is counted.
+// Column E of the chunk's row counts ids outside [0, E).
 __global__ void __launch_bounds__(kChunkThreads) k_hist(PlanArgs a) {
-  __shared__ int32_t sh[kMaxE];
+  __shared__ int32_t sh[kMaxE + 1];
   const int c = blockIdx.x, i = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
-  for (int e = tid; e < a.E; e += kChunkThreads) sh[e] = 0;
-  __syncthreads();
+  const int E = a.E;
+  for (int e = tid; e <= E; e += kChunkThreads) sh[e] = 0;
   const int64_t nk = int64_t(a.S) * a.K;
   const int64_t start = int64_t(c) * kChunk;
   const int n = (nk - start) < kChunk ? int(nk - start) : kChunk;
   const int32_t* src = a.ids + int64_t(i) * nk + start;
+  int ids[kPerThread];
+#pragma unroll
+  for (int u = 0; u < kPerThread; ++u) {
+    const int t = tid + u * kChunkThreads;
+    ids[u] = t < n ? __ldg(src + t) : -1;
+  }
+  __syncthreads();
   int bad = 0;
-  for (int t0 = 0; t0 < n; t0 += kChunkThreads) {  // warp-uniform trip count
-    const int t = t0 + tid;
-    const bool valid = t < n;
-    const int e = valid ? __ldg(src + t) : -1;
-    const bool ok = valid && e >= 0 && e < a.E;
-    bad += (valid && !ok);
+#pragma unroll
+  for (int u = 0; u < kPerThread; ++u) {
+    const int t = tid + u * kChunkThreads;
+    const int e = ids[u];
+    const bool ok = t < n && e >= 0 && e < E;
+    bad += (t < n && !ok);
     const unsigned peers = __match_any_sync(kFull, ok ? e : -1);
     if (ok && lane == __ffs(peers) - 1) atomicAdd(&sh[e], __popc(peers));
   }
-  bad = warp_sum(bad);
-  if (lane == 0 && bad) atomicAdd(&a.flags[kFlagBadIds], bad);
+  bad = int(__reduce_add_sync(kFull, unsigned(bad)));
+  if (lane == 0 && bad) atomicAdd(&sh[E], bad);
   __syncthreads();
-  int32_t* out = a.chunk_hist + (int64_t(i) * a.nchunk + c) * a.E;
-  for (int e = tid; e < a.E; e += kChunkThreads) {
-    const int v = sh[e];
-    out[e] = v;
-    if (v) atomicAdd(&a.cnt[i * a.E + e], v);
-  }
+  int32_t* out = a.chunk_hist + (int64_t(i) * a.nchunk + c) * (E + 1);
+  for (int e = tid; e <= E; e += kChunkThreads) out[e] = sh[e];
 }
 
 // ------------------------------------------------------------------ step 2+3
@@ -101,9 +104,10 @@ struct PlannerSmem {
   int32_t* repq;   // [P*R]
   int32_t* cu;     // [P*(Eh+R+1)]
   int32_t* hoff;   // [E+1]
-  int32_t* M;      // [warps][32 hosts][32 sources]
+  int32_t* order;  // [E]   experts with replicas first, then the rest
   int32_t* q;      // [warps][32 hosts] remaining quota in transport
   int32_t* misc;   // [16]
+  int32_t* M;      // [warps][32 hosts][32 sources]
 };
 
 __device__ PlannerSmem carve(char* base, const PlanArgs& a) {
@@ -116,23 +120,21 @@ __device__ PlannerSmem carve(char* base, const PlanArgs& a) {
   s.repq = p; p += a.P * a.R;
   s.cu = p; p += a.P * (a.Eh + a.R + 1);
   s.hoff = p; p += a.E + 1;
+  s.order = p; p += a.E;
   s.q = p; p += kPlanWarps * 32;
   s.misc = p; p += 16;
   s.M = p;
   return s;
 }
 
-enum { kMiscT = 0, kMiscMax = 1, kMiscNrep = 2, kMiscIters = 3, kMiscStatus = 4, kMiscErr = 5 };
+enum { kMiscT = 0, kMiscMax = 1, kMiscNrep = 2, kMiscIters = 3, kMiscBad = 4, kMiscErr = 5 };
 
 // Greedy replica placement, run by one warp; lane r holds rank r's load,
-// filled-slot count and stuck flag.  (ISER-MoE HALO-Q Objective 1 and stages
-// 2-3; Zepp 4.1 R slots per GPU and node-first hierarchical placement.)
-__device__ void greedy_warp(const PlanArgs& a, PlannerSmem& s, int T, int lane) {
+// filled-slot count and stuck flag, and every decision is one or two warp
+// reductions.  (ISER-MoE HALO-Q Objective 1 and stages 2-3; Zepp 4.1 R slots
+// per GPU and node-first hierarchical placement.)
+__device__ void greedy_warp(const PlanArgs& a, PlannerSmem& s, int T, int load, int lane) {
   const int P = a.P, R = a.R, Eh = a.Eh, gpn = a.gpn;
-  int load = 0;
-  if (lane < P) {
-    for (int e = lane * Eh; e < (lane + 1) * Eh; ++e) load += s.hq[e];
-  }
   int nfill = 0;
   bool stuck = lane >= P;
   int iters = 0;
@@ -142,45 +144,43 @@ __device__ void greedy_warp(const PlanArgs& a, PlannerSmem& s, int T, int lane) 
       gpn >= 32 ? kFull : (((1u << gpn) - 1u) << ((lane / gpn) * gpn));
   for (int guard = 0; guard <= max_iters; ++guard) {
     // donor: the busiest non-stuck rank, ties to the lowest rank
-    const unsigned long long dkey =
-        stuck ? 0ull : ((unsigned long long)(unsigned)(load + 1) << 5) | unsigned(31 - lane);
-    const unsigned long long dbest = warp_max_u64(dkey);
-    if (dbest == 0ull) break;
-    const int d = 31 - int(dbest & 31u);
-    const int dload = int(dbest >> 5) - 1;
+    const unsigned dl = stuck ? 0u : unsigned(load) + 1u;
+    const unsigned dmax = __reduce_max_sync(kFull, dl);
+    if (dmax == 0u) break;
+    const int d = __ffs(__ballot_sync(kFull, dl == dmax)) - 1;
+    const int dload = int(dmax - 1u);
     if (dload <= T) break;
     ++iters;
     // receivers with room: not the donor, a free slot, load below T
     const unsigned base = __ballot_sync(kFull, lane < P && lane != d && nfill < R && load < T);
-    // heaviest home expert of d (largest remaining quota, ties: lowest id)
-    // that has an eligible receiver, i.e. a rank in base without a copy
-    unsigned long long ebest = 0ull;
+    // d's heaviest home expert (largest remaining quota, ties: lowest id)
+    // that some rank in base can take (it holds no copy yet)
+    unsigned bq = 0u, bx = 0xffffffffu;
     for (int x = lane; x < Eh; x += 32) {
       const int e = d * Eh + x;
-      const int q = s.hq[e];
-      if (q > 0 && (base & ~s.hold[e]) != 0u) {
-        const unsigned long long k =
-            ((unsigned long long)(unsigned)q << 32) | (0xffffffffu - unsigned(x));
-        ebest = k > ebest ? k : ebest;
+      const unsigned q = unsigned(s.hq[e]);
+      if (q > 0u && (base & ~s.hold[e]) != 0u && q > bq) {
+        bq = q;
+        bx = unsigned(x);
       }
     }
-    ebest = warp_max_u64(ebest);
-    if (ebest == 0ull) {
+    const unsigned qmax = __reduce_max_sync(kFull, bq);
+    if (qmax == 0u) {
       if (lane == d) stuck = true;
       continue;
     }
-    const int e = d * Eh + int(0xffffffffu - unsigned(ebest & 0xffffffffu));
-    const int q = int(ebest >> 32);
+    const unsigned xmin = __reduce_min_sync(kFull, bq == qmax ? bx : 0xffffffffu);
+    const int e = d * Eh + int(xmin);
+    const int q = int(qmax);
     const unsigned hold = s.hold[e];
+    // receiver: a node without the expert first, then the lowest load, then
+    // the lowest rank
     const bool elig = ((base >> lane) & 1u) && !((hold >> lane) & 1u);
     const bool cov = ((e / Eh) / gpn == lane / gpn) || ((hold & node_mask) != 0u);
-    const unsigned long long rkey =
-        elig ? (((unsigned long long)cov << 40) | ((unsigned long long)(unsigned)load << 5) |
-                unsigned(lane))
-             : ~0ull;
-    const unsigned long long rbest = warp_min_u64(rkey);
-    const int r = int(rbest & 31u);
-    const int rload = int((rbest >> 5) & 0x7fffffffull);
+    const unsigned rk = elig ? (unsigned(load) | (cov ? 0x80000000u : 0u)) : 0xffffffffu;
+    const unsigned rmin = __reduce_min_sync(kFull, rk);
+    const int r = __ffs(__ballot_sync(kFull, elig && rk == rmin)) - 1;
+    const int rload = int(rmin & 0x7fffffffu);
     int m = dload - T;
     m = min(m, T - rload);
     m = min(m, q);
@@ -198,10 +198,8 @@ __device__ void greedy_warp(const PlanArgs& a, PlannerSmem& s, int T, int lane) 
     __syncwarp();
   }
   if (lane < P) a.load_after[lane] = load;
-  int mx = lane < P ? load : 0;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(kFull, mx, o));
-  const int nrep = warp_sum(lane < P ? nfill : 0);
+  const int mx = int(__reduce_max_sync(kFull, lane < P ? unsigned(load) : 0u));
+  const int nrep = int(__reduce_add_sync(kFull, lane < P ? unsigned(nfill) : 0u));
   if (lane == 0) {
     s.misc[kMiscMax] = mx;
     s.misc[kMiscNrep] = nrep;
@@ -209,37 +207,151 @@ __device__ void greedy_warp(const PlanArgs& a, PlannerSmem& s, int T, int lane) 
   }
 }
 
+// Transport of eq. (1) for expert e, run by one warp, lane = source rank.
+// Writes source lane's segments of e into the segment table and returns the
+// lane's share of the locality cost.
+__device__ long long transport_warp(const PlanArgs& a, PlannerSmem& s, int e, int lane,
+                                    int32_t* Mw, int32_t* qw) {
+  const int P = a.P, R = a.R, Eh = a.Eh, G = Eh + R, gpn = a.gpn;
+  const int h0 = e / Eh;
+  const unsigned hold = s.hold[e];
+  const int d = lane < P ? s.cnt[lane * a.E + e] : 0;
+  int2* seg = a.seg + int64_t(lane) * a.seg_width + s.hoff[e];
+  if (hold == 0u) {
+    // the home rank is the only host: every source sends it all its rows
+    const int inc = warp_incl_scan(d, lane);
+    if (lane < P)
+      seg[0] = make_int2(d, h0 * a.cap + s.cu[h0 * (G + 1) + (e - h0 * Eh)] + inc - d);
+    return (long long)cost_a(lane, h0, gpn) * d;
+  }
+  const unsigned hostmask = hold | (1u << h0);
+  const int nh = __popc(hostmask);
+  int dres = d;
+  for (int t = 0; t < nh; ++t) Mw[t * 32 + lane] = 0;
+  __syncwarp();
+  if (lane < P && ((hostmask >> lane) & 1u)) {
+    int q = 0;
+    if (lane == h0) {
+      q = s.hq[e];
+    } else {
+      for (int r = 0; r < R; ++r)
+        if (s.repe[lane * R + r] == e) q = s.repq[lane * R + r];
+    }
+    const int my_t = __popc(hostmask & ((1u << lane) - 1u));
+    const int take = min(dres, q);  // phase 0: the host's own rank, a = 0
+    Mw[my_t * 32 + lane] = take;
+    dres -= take;
+    qw[my_t] = q - take;
+  }
+  __syncwarp();
+  const int nlev = gpn > 1 ? 2 : 1;
+  for (int l = 0; l < nlev; ++l) {
+    const int lev = l == 0 ? 1 : 4;
+    unsigned hm = hostmask;
+    for (int t = 0; t < nh; ++t) {
+      const int j = __ffs(hm) - 1;
+      hm &= hm - 1u;
+      const int rem = qw[t];
+      const int v = (lane < P && cost_a(lane, j, gpn) == lev) ? dres : 0;
+      const int inc = warp_incl_scan(v, lane);
+      const int take = max(0, min(v, rem - (inc - v)));
+      const int tot = int(__reduce_add_sync(kFull, unsigned(take)));
+      Mw[t * 32 + lane] += take;
+      dres -= take;
+      __syncwarp();
+      if (lane == 0) qw[t] = rem - tot;
+      __syncwarp();
+    }
+  }
+  if (__any_sync(kFull, dres != 0) && lane == 0) atomicExch(&s.misc[kMiscErr], 1);
+  long long cost = 0;
+  {
+    unsigned hm = hostmask;
+    for (int t = 0; t < nh; ++t) {
+      const int j = __ffs(hm) - 1;
+      hm &= hm - 1u;
+      const int m = Mw[t * 32 + lane];
+      cost += (long long)cost_a(lane, j, gpn) * m;
+      const int inc = warp_incl_scan(m, lane);
+      __syncwarp();
+      Mw[t * 32 + lane] = inc;  // inclusive prefix over sources
+    }
+    __syncwarp();
+  }
+  if (lane < P) {
+    int idx = 0, cum = 0;
+    for (int lv = 0; lv < 3; ++lv) {
+      const int want = lv == 0 ? 0 : (lv == 1 ? 1 : 4);
+      unsigned hm = hostmask;
+      for (int t = 0; t < nh; ++t) {
+        const int j = __ffs(hm) - 1;
+        hm &= hm - 1u;
+        if (cost_a(lane, j, gpn) != want) continue;
+        const int inc = Mw[t * 32 + lane];
+        const int prev = lane > 0 ? Mw[t * 32 + lane - 1] : 0;
+        int grp;
+        if (j == h0) {
+          grp = e - h0 * Eh;
+        } else {
+          grp = Eh;
+          for (int r = 0; r < R; ++r)
+            if (s.repe[j * R + r] == e) grp = Eh + r;
+        }
+        cum += inc - prev;
+        seg[idx++] = make_int2(cum, j * a.cap + s.cu[j * (G + 1) + grp] + prev);
+      }
+    }
+  }
+  __syncwarp();
+  return cost;
+}
+
 __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
   extern __shared__ __align__(16) char smem_raw[];
+  __shared__ unsigned long long s_cost;
   PlannerSmem s = carve(smem_raw, a);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int P = a.P, E = a.E, R = a.R, Eh = a.Eh, G = Eh + R;
 
-  const int bad = a.flags[kFlagBadIds];
+  // route counts cnt[i][e] (and ids outside [0, E)) summed over the chunks
+  if (tid == 0) {
+    s.misc[kMiscBad] = 0;
+    s.misc[kMiscErr] = 0;
+    s_cost = 0ull;
+  }
+  __syncthreads();
+  for (int x = tid; x < P * (E + 1); x += kPlanThreads) {
+    const int i = x / (E + 1), e = x - i * (E + 1);
+    const int v = strided_sum(a.chunk_hist + int64_t(i) * a.nchunk * (E + 1) + e, a.nchunk,
+                              E + 1);
+    if (e < E) {
+      s.cnt[i * E + e] = v;
+      a.cnt[i * E + e] = v;
+    } else if (v) {
+      atomicAdd(&s.misc[kMiscBad], v);
+    }
+  }
+  for (int x = tid; x < P * R; x += kPlanThreads) {
+    s.repe[x] = -1;
+    s.repq[x] = 0;
+  }
+  __syncthreads();
+  const int bad = s.misc[kMiscBad];
   if (bad) {
     if (tid == 0) {
+      for (int k = 0; k < ZB_STATS_LEN; ++k) a.stats[k] = 0;
       a.stats[ZB_STAT_STATUS] = ZB_ERR_BAD_ID;
       a.stats[ZB_STAT_BAD_IDS] = bad;
-      for (int k = 1; k < ZB_STATS_LEN; ++k)
-        if (k != ZB_STAT_BAD_IDS) a.stats[k] = 0;
     }
     return;
   }
-
-  // T_e and the initial home quotas
-  for (int x = tid; x < P * E; x += kPlanThreads) s.cnt[x] = a.cnt[x];
-  __syncthreads();
+  // T_e, the initial home quotas
   for (int e = tid; e < E; e += kPlanThreads) {
     int t = 0;
     for (int i = 0; i < P; ++i) t += s.cnt[i * E + e];
     s.hq[e] = t;
     s.hold[e] = 0u;
   }
-  for (int x = tid; x < P * R; x += kPlanThreads) {
-    s.repe[x] = -1;
-    s.repq[x] = 0;
-  }
-  if (tid == 0) s.misc[kMiscErr] = 0;
   __syncthreads();
 
   if (warp == 0) {
@@ -251,13 +363,12 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
     const long long total = warp_sum64(lane < P ? (long long)L : 0ll);
     const int T = int((total + P - 1) / P);
     if (lane == 0) s.misc[kMiscT] = T;
-    greedy_warp(a, s, T, lane);
+    greedy_warp(a, s, T, L, lane);
   }
   __syncthreads();
 
   const int T = s.misc[kMiscT];
   const int max_load = s.misc[kMiscMax];
-  // plan tables
   for (int e = tid; e < E; e += kPlanThreads) a.home_quota[e] = s.hq[e];
   for (int x = tid; x < P * R; x += kPlanThreads) {
     a.rep_expert[x] = s.repe[x];
@@ -274,6 +385,18 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
       carry += __shfl_sync(kFull, inc, 31);
     }
     if (lane == 0) s.hoff[E] = carry;
+    // transport order: experts with replicas (the long case) first, so that
+    // they land on different warps, then the experts served by home alone
+    int n = 0;
+    for (int pass = 0; pass < 2; ++pass) {
+      for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        const bool take = e < E && ((s.hold[e] != 0u) == (pass == 0));
+        const unsigned m = __ballot_sync(kFull, take);
+        if (take) s.order[n + __popc(m & ((1u << lane) - 1u))] = e;
+        n += __popc(m);
+      }
+    }
   }
   // cu_seqlens: exclusive prefix of each rank's group receipts (exact quotas)
   for (int j = warp; j < P; j += kPlanWarps) {
@@ -296,101 +419,12 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
   const bool capacity = max_load > a.cap;
   long long cost_part = 0;
   if (!capacity) {
-    // Transport of eq. (1), one warp per expert, lane = source rank.
     int32_t* Mw = s.M + warp * 32 * 32;
     int32_t* qw = s.q + warp * 32;
-    for (int e = warp; e < E; e += kPlanWarps) {
-      const int h0 = e / Eh;
-      const unsigned hostmask = s.hold[e] | (1u << h0);
-      const int nh = __popc(hostmask);
-      int dres = lane < P ? s.cnt[lane * E + e] : 0;
-      // host index of lane's own rank, its quota and group
-      const bool is_host = lane < P && ((hostmask >> lane) & 1u);
-      const int my_t = __popc(hostmask & ((1u << lane) - 1u));
-      for (int t = 0; t < nh; ++t) Mw[t * 32 + lane] = 0;
-      __syncwarp();
-      if (is_host) {
-        int q = 0;
-        if (lane == h0) {
-          q = s.hq[e];
-        } else {
-          for (int r = 0; r < R; ++r)
-            if (s.repe[lane * R + r] == e) q = s.repq[lane * R + r];
-        }
-        const int take = min(dres, q);  // phase 0: the host's own rank, a = 0
-        Mw[my_t * 32 + lane] = take;
-        dres -= take;
-        qw[my_t] = q - take;
-      }
-      __syncwarp();
-      const int nlev = a.gpn > 1 ? 2 : 1;
-      for (int l = 0; l < nlev; ++l) {
-        const int lev = l == 0 ? 1 : 4;
-        unsigned hm = hostmask;
-        for (int t = 0; t < nh; ++t) {
-          const int j = __ffs(hm) - 1;
-          hm &= hm - 1u;
-          const int rem = qw[t];
-          const bool el = lane < P && cost_a(lane, j, a.gpn) == lev;
-          const int v = el ? dres : 0;
-          const int inc = warp_incl_scan(v, lane);
-          const int take = max(0, min(v, rem - (inc - v)));
-          const int tot = warp_sum(take);
-          Mw[t * 32 + lane] += take;
-          dres -= take;
-          __syncwarp();
-          if (lane == 0) qw[t] = rem - tot;
-          __syncwarp();
-        }
-      }
-      if (warp_sum(dres != 0) != 0 && lane == 0) atomicExch(&s.misc[kMiscErr], 1);
-      // locality cost, segment starts and the segment table of each source
-      {
-        unsigned hm = hostmask;
-        for (int t = 0; t < nh; ++t) {
-          const int j = __ffs(hm) - 1;
-          hm &= hm - 1u;
-          const int m = Mw[t * 32 + lane];
-          cost_part += (long long)cost_a(lane, j, a.gpn) * m;
-          const int inc = warp_incl_scan(m, lane);
-          __syncwarp();
-          Mw[t * 32 + lane] = inc;  // inclusive prefix over sources
-        }
-        __syncwarp();
-      }
-      if (lane < P) {
-        int2* seg = a.seg + int64_t(lane) * a.seg_width + s.hoff[e];
-        int idx = 0, cum = 0;
-        for (int lv = 0; lv < 3; ++lv) {
-          const int want = lv == 0 ? 0 : (lv == 1 ? 1 : 4);
-          unsigned hm = hostmask;
-          for (int t = 0; t < nh; ++t) {
-            const int j = __ffs(hm) - 1;
-            hm &= hm - 1u;
-            if (cost_a(lane, j, a.gpn) != want) continue;
-            const int inc = Mw[t * 32 + lane];
-            const int prev = lane > 0 ? Mw[t * 32 + lane - 1] : 0;
-            int grp;
-            if (j == h0) {
-              grp = e - h0 * Eh;
-            } else {
-              grp = Eh;
-              for (int r = 0; r < R; ++r)
-                if (s.repe[j * R + r] == e) grp = Eh + r;
-            }
-            cum += inc - prev;
-            const int base = j * a.cap + s.cu[j * (G + 1) + grp] + prev;
-            seg[idx++] = make_int2(cum, base);
-          }
-        }
-      }
-      __syncwarp();
-    }
+    for (int k = warp; k < E; k += kPlanWarps)
+      cost_part += transport_warp(a, s, s.order[k], lane, Mw, qw);
   }
   cost_part = warp_sum64(cost_part);
-  __shared__ unsigned long long s_cost;
-  if (tid == 0) s_cost = 0ull;
-  __syncthreads();
   if (lane == 0) atomicAdd(&s_cost, (unsigned long long)cost_part);
   __syncthreads();
   if (tid == 0) {
@@ -398,7 +432,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
     if (capacity)
       status = ZB_ERR_CAPACITY;
     else if (s.misc[kMiscErr])
-      status = ZB_ERR_INVALID;  // unreachable: transport always closes
+      status = ZB_ERR_INVALID;  // unreachable: the transport always closes
     else if (max_load > T)
       status = ZB_WARN_UNBALANCED;
     a.stats[ZB_STAT_STATUS] = status;
@@ -415,11 +449,16 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
 // ------------------------------------------------------------------ step 3
 
 constexpr int kAssignWarps = kChunkThreads / 32;
-constexpr int kPerWarp = kChunk / kAssignWarps;  // 256 entries, 8 steps of 32
+constexpr int kPerWarp = kChunk / kAssignWarps;  // kPerThread steps of 32
 
+// One CTA per (chunk c, source rank i).  Warp w owns entries
+// [kPerWarp*w, kPerWarp*(w+1)) of the chunk and walks them 32 at a time in flat
+// order, so ranks among equal experts come out in flat-index order.
 __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
   if (a.stats[ZB_STAT_STATUS] < 0) return;  // bad ids or capacity: no rows
   __shared__ int32_t wh[kAssignWarps][kMaxE];  // per-warp running position
+  __shared__ int32_t s_hoff[kMaxE + 1];
+  __shared__ int2 s_seg[kMaxSegWidth];
   const int c = blockIdx.x, i = blockIdx.y, tid = threadIdx.x, lane = tid & 31,
             warp = tid >> 5;
   const int E = a.E;
@@ -427,23 +466,31 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
   const int64_t start = int64_t(c) * kChunk;
   const int n = (nk - start) < kChunk ? int(nk - start) : kChunk;
   const int32_t* src = a.ids + int64_t(i) * nk + start;
+  const int w0 = warp * kPerWarp;
+  int ids[kPerThread];
+#pragma unroll
+  for (int u = 0; u < kPerThread; ++u) {
+    const int t = w0 + 32 * u + lane;
+    ids[u] = t < n ? __ldg(src + t) : -1;
+  }
+  for (int x = tid; x < kAssignWarps * kMaxE; x += kChunkThreads) (&wh[0][0])[x] = 0;
+  for (int e = tid; e <= E; e += kChunkThreads) s_hoff[e] = a.hoff[e];
+  const int2* segrow = a.seg + int64_t(i) * a.seg_width;
+  for (int x = tid; x < a.seg_width; x += kChunkThreads) s_seg[x] = segrow[x];
+  __syncthreads();
 
   // pass 1: per-warp histogram of the warp's slice
-  for (int x = tid; x < kAssignWarps * kMaxE; x += kChunkThreads) (&wh[0][0])[x] = 0;
-  __syncthreads();
-  const int w0 = warp * kPerWarp;
-  for (int t0 = 0; t0 < kPerWarp; t0 += 32) {
-    const int t = w0 + t0 + lane;
-    const int e = t < n ? __ldg(src + t) : -1;
+#pragma unroll
+  for (int u = 0; u < kPerThread; ++u) {
+    const int e = ids[u];
     const unsigned peers = __match_any_sync(kFull, e);
     if (e >= 0 && lane == __ffs(peers) - 1) wh[warp][e] += __popc(peers);
   }
   __syncthreads();
   // exclusive prefix: earlier chunks of this source, then earlier warps
   for (int e = tid; e < E; e += kChunkThreads) {
-    int run = 0;
-    const int32_t* ch = a.chunk_hist + int64_t(i) * a.nchunk * E + e;
-    for (int cc = 0; cc < c; ++cc) run += ch[int64_t(cc) * E];
+    int run = strided_sum(a.chunk_hist + int64_t(i) * a.nchunk * (E + 1) + e, c, E + 1);
+#pragma unroll
     for (int w = 0; w < kAssignWarps; ++w) {
       const int v = wh[w][e];
       wh[w][e] = run;
@@ -452,10 +499,10 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
   }
   __syncthreads();
   // pass 2: stable position of each entry, then its segment and row
-  const int2* segrow = a.seg + int64_t(i) * a.seg_width;
-  for (int t0 = 0; t0 < kPerWarp; t0 += 32) {
-    const int t = w0 + t0 + lane;
-    const int e = t < n ? __ldg(src + t) : -1;
+  const int64_t nrows = int64_t(a.P) * a.cap;
+#pragma unroll
+  for (int u = 0; u < kPerThread; ++u) {
+    const int e = ids[u];
     const unsigned peers = __match_any_sync(kFull, e);
     int p = 0;
     if (e >= 0) p = wh[warp][e] + __popc(peers & ((1u << lane) - 1u));
@@ -463,20 +510,19 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
     if (e >= 0 && lane == __ffs(peers) - 1) wh[warp][e] += __popc(peers);
     __syncwarp();
     if (e >= 0) {
-      const int h_begin = a.hoff[e], h_end = a.hoff[e + 1];
+      const int h_end = s_hoff[e + 1];
       int prev = 0, row = -1;
-      for (int h = h_begin; h < h_end; ++h) {
-        const int2 sg = segrow[h];
+      for (int h = s_hoff[e]; h < h_end; ++h) {
+        const int2 sg = s_seg[h];
         if (p < sg.x) {
           row = sg.y + (p - prev);
           break;
         }
         prev = sg.x;
       }
-      const int64_t g = int64_t(i) * nk + start + t;
+      const int64_t g = int64_t(i) * nk + start + w0 + 32 * u + lane;
       a.dst_row[g] = row;
-      if (a.row_src && row >= 0 && int64_t(row) < int64_t(a.P) * a.cap)
-        a.row_src[row] = int32_t(g);
+      if (a.row_src && row >= 0 && int64_t(row) < nrows) a.row_src[row] = int32_t(g);
     }
   }
 }
@@ -486,8 +532,8 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
 size_t planner_smem_bytes(const zb_config& c) {
   const int Eh = c.E / c.P;
   size_t words = size_t(c.P) * c.E + 2 * size_t(c.E) + 2 * size_t(c.P) * c.R +
-                 size_t(c.P) * (Eh + c.R + 1) + size_t(c.E + 1) + kPlanWarps * 32 + 16;
-  words = (words + 3) & ~size_t(3);
+                 size_t(c.P) * (Eh + c.R + 1) + size_t(c.E + 1) + size_t(c.E) +
+                 kPlanWarps * 32 + 16;
   words += size_t(kPlanWarps) * 32 * 32;
   return words * sizeof(int32_t);
 }

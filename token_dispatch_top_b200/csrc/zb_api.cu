@@ -83,15 +83,10 @@ int zb_plan(const zb_config* c, const int32_t* ids, const zb_plan_t* plan, void*
   a.home_quota = plan->home_quota; a.load_before = plan->load_before;
   a.load_after = plan->load_after; a.cu_seqlens = plan->cu_seqlens; a.dst_row = plan->dst_row;
   a.row_src = plan->row_src; a.stats = plan->stats;
-  a.flags = reinterpret_cast<int32_t*>(base + w.off_flags);
   a.chunk_hist = reinterpret_cast<int32_t*>(base + w.off_chunk_hist);
   a.hoff = reinterpret_cast<int32_t*>(base + w.off_hoff);
   a.seg = reinterpret_cast<int2*>(base + w.off_seg);
 
-  if (cudaMemsetAsync(a.flags, 0, sizeof(int32_t) * zb::kFlagWords, s) != cudaSuccess)
-    return ZB_ERR_CUDA;
-  if (cudaMemsetAsync(a.cnt, 0, sizeof(int32_t) * size_t(c->P) * c->E, s) != cudaSuccess)
-    return ZB_ERR_CUDA;
   if (a.row_src &&
       cudaMemsetAsync(a.row_src, 0xff, sizeof(int32_t) * size_t(c->P) * c->cap_rows, s) !=
           cudaSuccess)

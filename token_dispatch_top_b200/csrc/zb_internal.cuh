@@ -13,21 +13,22 @@ namespace zb {
 // Entries of one source rank handled by one CTA of the histogram and the
 // assignment kernels.
 constexpr int kChunk = 2048;
-constexpr int kChunkThreads = 256;
+constexpr int kChunkThreads = 512;
 constexpr int kMaxE = 384;
 constexpr int kMaxP = 32;
 constexpr int kPlanThreads = 512;  // 16 warps
 constexpr int kPlanWarps = kPlanThreads / 32;
 
-// Workspace flag words.
-enum { kFlagBadIds = 0, kFlagInternal = 1, kFlagWords = 64 };
+// Widest row of the segment table: E + P*R entries.
+constexpr int kMaxSegWidth = kMaxE + kMaxP * (kMaxP - 1);
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Layout of the scratch workspace (all offsets 256-byte aligned):
-//   flags      int32 [kFlagWords]
-//   chunk_hist int32 [P][nchunk][E]    per-chunk expert counts
+// Layout of the scratch workspace (all offsets 256-byte aligned).  Nothing in
+// it needs initialising: every word is written before it is read.
+//   chunk_hist int32 [P][nchunk][E+1]  per-chunk expert counts; column E
+//                                      counts the chunk's ids outside [0, E)
 //   hoff       int32 [E+1]             first segment of expert e in a row of seg
 //   seg        int2  [P][E + P*R]      per (source i, expert e): the hosts in
 //                                      the order source i fills them, as
@@ -35,7 +36,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct Workspace {
   int nchunk;
   int seg_width;
-  size_t off_flags, off_chunk_hist, off_hoff, off_seg, bytes;
+  size_t off_chunk_hist, off_hoff, off_seg, bytes;
 };
 
 inline Workspace workspace_layout(const zb_config& c) {
@@ -44,10 +45,8 @@ inline Workspace workspace_layout(const zb_config& c) {
   w.nchunk = int(ceil_div(nk, kChunk));
   w.seg_width = c.E + c.P * c.R;
   size_t o = 0;
-  w.off_flags = o;
-  o = align256(o + sizeof(int32_t) * kFlagWords);
   w.off_chunk_hist = o;
-  o = align256(o + sizeof(int32_t) * size_t(c.P) * w.nchunk * c.E);
+  o = align256(o + sizeof(int32_t) * size_t(c.P) * w.nchunk * (c.E + 1));
   w.off_hoff = o;
   o = align256(o + sizeof(int32_t) * size_t(c.E + 1));
   w.off_seg = o;
@@ -71,7 +70,6 @@ struct PlanArgs {
   int32_t* dst_row;
   int32_t* row_src;
   int64_t* stats;
-  int32_t* flags;
   int32_t* chunk_hist;
   int32_t* hoff;
   int2* seg;
