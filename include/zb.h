@@ -65,12 +65,25 @@ extern "C" {
  *   gpus_per_node  1 = flat locality cost; g > 1 groups ranks into nodes of g
  *       consecutive ranks (P % g == 0)
  *   cap_rows  rows of each rank's receive buffer, >= S*K; P*cap_rows and
- *       P*S*K must fit in int32 */
+ *       P*S*K must fit in int32
+ *   policy  receiver choice of the greedy planner:
+ *       ZB_POLICY_ROOM (0): among eligible ranks, the one whose node does not
+ *         yet hold the expert, then the lowest load, then the lowest rank;
+ *       ZB_POLICY_LOCAL (1): balance first, locality among equal moves:
+ *         after node coverage, the rank that takes the most rows m_r (the
+ *         move's balance progress), then the rank whose own rows for the
+ *         expert the copy would serve locally are most, min(cnt[r][e], m_r),
+ *         then the lowest load, then the lowest rank (ISER-MoE, HALO-Q
+ *         Objective 2: the most locally computed tokens among balanced
+ *         routings). */
+#define ZB_POLICY_ROOM 0
+#define ZB_POLICY_LOCAL 1
 typedef struct zb_config {
   int P, E, K, S, H, R;
   float C;
   int gpus_per_node;
   int cap_rows;
+  int policy;
 } zb_config;
 
 /* Indices into plan->stats (int64). */
@@ -136,9 +149,10 @@ ZB_API size_t zb_workspace_bytes(const zb_config *cfg);
  *    it offers its heaviest home expert (largest remaining home quota, ties:
  *    lowest expert) for which an eligible receiver exists; eligible = another
  *    rank with a free slot, load below T and no copy of the expert; the
- *    receiver is the one whose node does not yet hold the expert, then the
- *    lowest load, then the lowest rank (Zepp "4.1 Expert Placement and Token
- *    Routing": R extra slots per GPU, round-robin across nodes first); it takes
+ *    receiver is chosen by cfg->policy (see zb_config): by default the one
+ *    whose node does not yet hold the expert, then the lowest load, then the
+ *    lowest rank (Zepp "4.1 Expert Placement and Token Routing": R extra
+ *    slots per GPU, round-robin across nodes first); it takes
  *    m = min(load_d - T, T - load_r, quota_e) rows into its lowest free slot
  *    (HALO-Q stages 2-3).  A donor with no movable expert is marked stuck;
  *  - routing: expert e's rows are assigned to its hosts by eq. (1) of Zepp 4.1,

@@ -45,7 +45,7 @@ class _Cfg(ctypes.Structure):
     _fields_ = [("P", ctypes.c_int), ("E", ctypes.c_int), ("K", ctypes.c_int),
                 ("S", ctypes.c_int), ("H", ctypes.c_int), ("R", ctypes.c_int),
                 ("C", ctypes.c_double), ("gpus_per_node", ctypes.c_int),
-                ("cap_rows", ctypes.c_int)]
+                ("cap_rows", ctypes.c_int), ("policy", ctypes.c_int)]
 
 
 _P32 = ctypes.POINTER(ctypes.c_int32)
@@ -97,13 +97,14 @@ class Config:
     C: float = 0.0
     gpus_per_node: int = 1
     cap_rows: int | None = None
+    policy: int = 0  # receiver choice: 0 most room, 1 most local rows
 
     def cap(self) -> int:
         return self.S * self.K if self.cap_rows is None else self.cap_rows
 
     def c(self) -> _Cfg:
         return _Cfg(self.P, self.E, self.K, self.S, self.H, self.R, float(self.C),
-                    self.gpus_per_node, self.cap())
+                    self.gpus_per_node, self.cap(), self.policy)
 
 
 def _ptr(a: np.ndarray):

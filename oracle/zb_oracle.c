@@ -30,6 +30,11 @@
  *    lowest expert id; the receiver is the eligible rank with the most room
  *    (lowest load), ties to the lowest rank; with nodes, a rank on a node that
  *    does not yet hold the expert comes first (round-robin across nodes).
+ *    Policy 1 keeps balance first and breaks its ties by locality (ISER-MoE,
+ *    HALO-Q Objective 2: the most locally computed tokens among balanced
+ *    routings): after node coverage, the largest move m_r = min(load_d - T,
+ *    T - load_r, quota_e), then the most rows of the receiver's own demand
+ *    the copy would serve, min(cnt[r][e], m_r), then lowest load and rank.
  *  - quotas are delivered exactly (|sum_i M_ij - q_j| = 0 <= C*q_j), because
  *    T = S*K leaves no slack in the fixed S*K buffers.
  *  - rows inside a group are ordered by (source rank, flat index s*K+k).
@@ -61,6 +66,7 @@ typedef struct {
   double C;          /* relaxation ratio of eq. (1); validated, recorded */
   int gpus_per_node; /* 1 = flat locality cost; >1 = two-level cost */
   int cap_rows;      /* rows of each rank's receive buffer (>= S*K) */
+  int policy;        /* receiver choice: 0 most room, 1 most local rows */
 } zbo_config;
 
 typedef struct {
@@ -108,6 +114,7 @@ int zbo_validate(const zbo_config *c) {
   if (c->cap_rows < c->S * c->K) return ZBO_ERR_INVALID;
   if ((int64_t)c->P * c->S * c->K > INT32_MAX) return ZBO_ERR_INVALID;
   if ((int64_t)c->P * c->cap_rows > INT32_MAX) return ZBO_ERR_INVALID;
+  if (c->policy != 0 && c->policy != 1) return ZBO_ERR_INVALID;
   return ZBO_OK;
 }
 
@@ -157,12 +164,16 @@ static int node_covers(const slots_t *st, int r, int e) {
  * ISER stage 3].  Repeatedly: the busiest rank d (ties: lowest rank) offers
  * its heaviest home expert (largest remaining home quota, ties: lowest id)
  * that some rank can take; the receiver is the eligible rank with the most
- * room (node coverage first when there are nodes), and receives
+ * room (node coverage first when there are nodes; with policy 1, the largest
+ * move m_r, then the most rows of its own demand for the expert that the
+ * copy would serve locally, come before room: locality among equally
+ * balancing moves, after ISER-MoE's Objective 2), and receives
  * m = min(load[d]-T, T-load[r], hq[e]) of that expert's rows in its lowest
  * free slot.  A donor for which no expert has an eligible receiver is marked
  * stuck.  Stops when the busiest non-stuck rank is at or below T. */
-static void greedy_place(const zbo_config *c, int32_t T, int32_t *load, int32_t *hq,
-                         int32_t *rep_expert, int32_t *rep_quota, int32_t *n_iters) {
+static void greedy_place(const zbo_config *c, const int32_t *cnt, int32_t T, int32_t *load,
+                         int32_t *hq, int32_t *rep_expert, int32_t *rep_quota,
+                         int32_t *n_iters) {
   const int P = c->P, E = c->E, R = c->R, Eh = E / P;
   int *nfill = calloc((size_t)P, sizeof(int));
   int *stuck = calloc((size_t)P, sizeof(int));
@@ -190,12 +201,30 @@ static void greedy_place(const zbo_config *c, int32_t T, int32_t *load, int32_t 
     for (int t = 0; t < n && pick_e < 0; t++) {
       int e = order[t];
       int best = -1, best_cov = 0;
+      int32_t best_gain = 0, best_m = 0;
       for (int r = 0; r < P; r++) {
         if (r == d || nfill[r] >= R || load[r] >= T || holds_replica(&st, r, e)) continue;
         int cov = node_covers(&st, r, e);
-        if (best < 0 || cov < best_cov || (cov == best_cov && load[r] < load[best])) {
+        /* policy 1: the rows r would take (the move's balance progress), then
+         * the rows of r's own demand the copy would serve locally */
+        int32_t mr = 0, gain = 0;
+        if (c->policy == 1) {
+          mr = load[d] - T;
+          if (T - load[r] < mr) mr = T - load[r];
+          if (hq[e] < mr) mr = hq[e];
+          gain = cnt[(size_t)r * c->E + e] < mr ? cnt[(size_t)r * c->E + e] : mr;
+        }
+        int better;
+        if (best < 0) better = 1;
+        else if (cov != best_cov) better = cov < best_cov;
+        else if (mr != best_m) better = mr > best_m;
+        else if (gain != best_gain) better = gain > best_gain;
+        else better = load[r] < load[best];
+        if (better) {
           best = r;
           best_cov = cov;
+          best_m = mr;
+          best_gain = gain;
         }
       }
       if (best >= 0) { pick_e = e; pick_r = best; }
@@ -300,8 +329,8 @@ int zbo_plan(const zbo_config *c, const int32_t *ids, zbo_plan_out *out) {
   out->water_level = T;
 
   for (int e = 0; e < E; e++) out->home_quota[e] = Te[e];
-  greedy_place(c, T, out->load_after, out->home_quota, out->rep_expert, out->rep_quota,
-               &out->n_iters);
+  greedy_place(c, out->cnt, T, out->load_after, out->home_quota, out->rep_expert,
+               out->rep_quota, &out->n_iters);
 
   out->max_load = 0;
   out->n_replicas = 0;

@@ -57,6 +57,7 @@ def _both(**kw):
     dict(C=-0.5), dict(C=1.0), dict(C=0.99), dict(gpus_per_node=0), dict(gpus_per_node=3),
     dict(gpus_per_node=2), dict(cap_rows=127), dict(cap_rows=128), dict(P=32, E=384, R=31),
     dict(P=1, E=384, R=0), dict(K=16), dict(S=2 ** 27, K=16), dict(S=2 ** 26, K=8, P=8, E=16),
+    dict(policy=1), dict(policy=2), dict(policy=-1),
 ])
 def test_validation_agrees_with_oracle(lib, kw):
     c, o = _both(**kw)

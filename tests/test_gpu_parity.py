@@ -77,7 +77,8 @@ def full_parity(zc, oc, ids, w, hidden_bits, y_bits, dev, with_row_src=True, str
 def test_hand_examples(dev, ex):
     d = ex["cfg"]
     kw = dict(P=d["P"], E=d["E"], K=d["K"], S=d["S"], H=d["H"], R=d["R"],
-              gpus_per_node=d.get("gpus_per_node", 1), cap_rows=d.get("cap_rows"))
+              gpus_per_node=d.get("gpus_per_node", 1), cap_rows=d.get("cap_rows"),
+              policy=d.get("policy", 0))
     zc, oc = zb.Config(**kw), oracle.Config(**kw)
     ids = np.array(ex["ids"], np.int32).reshape(zc.P, zc.S, zc.K)
     rng = np.random.default_rng(0)
@@ -103,7 +104,8 @@ def _small_cases(n=60, seed=21):
         p = 1.0 / np.arange(1, E + 1) ** rng.uniform(0, 2)
         p = p[rng.permutation(E)] / p.sum()
         ids = rng.choice(E, size=(P, S, K), p=p).astype(np.int32)
-        out.append((dict(P=P, E=E, K=K, S=S, H=H, R=R, C=0.1, gpus_per_node=gpn), ids))
+        out.append((dict(P=P, E=E, K=K, S=S, H=H, R=R, C=0.1, gpus_per_node=gpn,
+                         policy=len(out) % 2), ids))
     return out
 
 
@@ -192,6 +194,17 @@ def sampled_data_parity(zc, oc, p, o, ids, w, hidden_d, dev, n=384, seed=0):
     got_o = bf16_to_bits(out.view(P * S, H).index_select(0, torch.from_numpy(tok).to(dev)))
     np.testing.assert_array_equal(got_o, want_o[0])
     del buf, y, out
+
+
+@pytest.mark.parametrize("name,seed", [("mid", 0), ("mid", 3), ("hot", 0), ("hot", 1),
+                                       ("hier", 0), ("hier", 2)])
+def test_locality_policy_plan(dev, name, seed):
+    """The locality-aware receiver policy, full-size plans bit-exact."""
+    wl = synth.WORKLOADS[name]
+    zc, oc = cfgs(wl, cap_rows=2 * wl.S * wl.K, policy=zb.POLICY_LOCAL)
+    ids, _ = synth.routing(wl, seed)
+    p, status, _ = gpu_plan(zc, ids, dev, with_row_src=False)
+    assert_plan_equal(plan_tables(p), oracle.plan(oc, ids, want_M=False), status)
 
 
 @pytest.mark.parametrize("name", ["hot", "hier"])

@@ -21,7 +21,7 @@ GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_examples.json")
 def _cfg(d):
     return oracle.Config(P=d["P"], E=d["E"], K=d["K"], S=d["S"], H=d["H"], R=d["R"],
                          C=d.get("C", 0.0), gpus_per_node=d.get("gpus_per_node", 1),
-                         cap_rows=d.get("cap_rows"))
+                         cap_rows=d.get("cap_rows"), policy=d.get("policy", 0))
 
 
 def _examples():
@@ -55,7 +55,7 @@ def test_hand_examples(ex):
 
 # ---------------------------------------------------------------- random cases
 
-def _random_case(rng, P, Eh, K, S, R, gpn=1, skew=1.5, cap_extra=None):
+def _random_case(rng, P, Eh, K, S, R, gpn=1, skew=1.5, cap_extra=None, policy=0):
     E = P * Eh
     p = 1.0 / np.arange(1, E + 1) ** skew
     p = p[rng.permutation(E)] if rng.random() < 0.5 else p
@@ -64,7 +64,7 @@ def _random_case(rng, P, Eh, K, S, R, gpn=1, skew=1.5, cap_extra=None):
     ids = rng.choice(E, size=(P, S, K), p=p).astype(np.int32)
     cap = None if cap_extra is None else S * K + cap_extra
     return oracle.Config(P=P, E=E, K=K, S=S, H=8, R=R, C=0.1, gpus_per_node=gpn,
-                         cap_rows=cap), ids
+                         cap_rows=cap, policy=policy), ids
 
 
 def _cases(n=120, seed=7):
@@ -80,7 +80,7 @@ def _cases(n=120, seed=7):
         S = int(rng.integers(0, 12))
         R = int(rng.integers(0, P)) if P > 1 else 0
         out.append(_random_case(rng, P, Eh, K, S, R, gpn, skew=float(rng.uniform(0, 2.5)),
-                                cap_extra=10 ** 6))
+                                cap_extra=10 ** 6, policy=t % 2))
     return out
 
 
@@ -267,7 +267,8 @@ def test_degenerate_shapes():
 def test_errors():
     ids = np.zeros((2, 2, 1), np.int32)
     for bad in [dict(P=0), dict(E=3), dict(E=400), dict(K=0), dict(K=17), dict(H=12), dict(H=0),
-                dict(R=2), dict(R=-1), dict(C=1.0), dict(C=-0.1), dict(gpus_per_node=3)]:
+                dict(R=2), dict(R=-1), dict(C=1.0), dict(C=-0.1), dict(gpus_per_node=3),
+                dict(policy=2), dict(policy=-1)]:
         d = dict(P=2, E=4, K=1, S=2, H=8, R=1, C=0.0, gpus_per_node=1)
         d.update(bad)
         assert oracle.validate(oracle.Config(**d)) == oracle.ERR_INVALID, bad

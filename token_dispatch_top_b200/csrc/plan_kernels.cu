@@ -177,10 +177,30 @@ __device__ void greedy_warp(const PlanArgs& a, PlannerSmem& s, int T, int load, 
     // the lowest rank
     const bool elig = ((base >> lane) & 1u) && !((hold >> lane) & 1u);
     const bool cov = ((e / Eh) / gpn == lane / gpn) || ((hold & node_mask) != 0u);
-    const unsigned rk = elig ? (unsigned(load) | (cov ? 0x80000000u : 0u)) : 0xffffffffu;
-    const unsigned rmin = __reduce_min_sync(kFull, rk);
-    const int r = __ffs(__ballot_sync(kFull, elig && rk == rmin)) - 1;
-    const int rload = int(rmin & 0x7fffffffu);
+    int r, rload;
+    if (a.policy == ZB_POLICY_LOCAL) {
+      // balance first, locality among equal moves (HALO-Q Objective 2): after
+      // node coverage, the largest move m_r, then the most own rows the copy
+      // would serve locally, min(cnt[r][e], m_r), then load and rank
+      const int mr = min(min(dload - T, T - load), q);
+      const int own = lane < P ? s.cnt[lane * a.E + e] : 0;
+      const int gain = min(own, mr);
+      const unsigned k1 =
+          elig ? ((cov ? 0x80000000u : 0u) | unsigned(0x7fffffff - mr)) : 0xffffffffu;
+      const unsigned k1min = __reduce_min_sync(kFull, k1);
+      const bool c1 = elig && k1 == k1min;
+      const unsigned k2 = c1 ? unsigned(0x7fffffff - gain) : 0xffffffffu;
+      const unsigned k2min = __reduce_min_sync(kFull, k2);
+      const bool c2 = c1 && k2 == k2min;
+      const unsigned lmin = __reduce_min_sync(kFull, c2 ? unsigned(load) : 0xffffffffu);
+      r = __ffs(__ballot_sync(kFull, c2 && unsigned(load) == lmin)) - 1;
+      rload = int(lmin);
+    } else {
+      const unsigned rk = elig ? (unsigned(load) | (cov ? 0x80000000u : 0u)) : 0xffffffffu;
+      const unsigned rmin = __reduce_min_sync(kFull, rk);
+      r = __ffs(__ballot_sync(kFull, elig && rk == rmin)) - 1;
+      rload = int(rmin & 0x7fffffffu);
+    }
     int m = dload - T;
     m = min(m, T - rload);
     m = min(m, q);

@@ -56,6 +56,7 @@ int zb_validate(const zb_config* c) {
   if (int64_t(c->cap_rows) < sk) return ZB_ERR_INVALID;
   if (int64_t(c->P) * sk > INT32_MAX) return ZB_ERR_INVALID;
   if (int64_t(c->P) * c->cap_rows > INT32_MAX) return ZB_ERR_INVALID;
+  if (c->policy != ZB_POLICY_ROOM && c->policy != ZB_POLICY_LOCAL) return ZB_ERR_INVALID;
   return ZB_OK;
 }
 
@@ -76,7 +77,7 @@ int zb_plan(const zb_config* c, const int32_t* ids, const zb_plan_t* plan, void*
 
   zb::PlanArgs a{};
   a.P = c->P; a.E = c->E; a.K = c->K; a.S = c->S; a.R = c->R; a.Eh = c->E / c->P;
-  a.gpn = c->gpus_per_node; a.cap = c->cap_rows;
+  a.gpn = c->gpus_per_node; a.cap = c->cap_rows; a.policy = c->policy;
   a.nchunk = w.nchunk; a.seg_width = w.seg_width;
   a.ids = ids;
   a.cnt = plan->cnt; a.rep_expert = plan->rep_expert; a.rep_quota = plan->rep_quota;

@@ -57,7 +57,7 @@ inline Workspace workspace_layout(const zb_config& c) {
 
 // Kernel parameter block shared by the plan kernels.
 struct PlanArgs {
-  int P, E, K, S, R, Eh, gpn, cap;
+  int P, E, K, S, R, Eh, gpn, cap, policy;
   int nchunk, seg_width;
   const int32_t* ids;
   int32_t* cnt;

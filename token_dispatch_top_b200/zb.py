@@ -25,6 +25,9 @@ ERR_BAD_ID = -3
 ERR_TIMEOUT = -4
 ERR_CUDA = -5
 
+POLICY_ROOM = 0   # receiver with the most room (after node coverage)
+POLICY_LOCAL = 1  # the largest move, then the most rows served locally
+
 STAT_STATUS, STAT_MAX_LOAD, STAT_N_REPLICAS, STAT_N_ITERS, STAT_WATER_LEVEL, \
     STAT_LOCALITY_COST, STAT_BAD_IDS = range(7)
 STATS_LEN = 8
@@ -43,7 +46,7 @@ class _Cfg(ctypes.Structure):
     _fields_ = [("P", ctypes.c_int), ("E", ctypes.c_int), ("K", ctypes.c_int),
                 ("S", ctypes.c_int), ("H", ctypes.c_int), ("R", ctypes.c_int),
                 ("C", ctypes.c_float), ("gpus_per_node", ctypes.c_int),
-                ("cap_rows", ctypes.c_int)]
+                ("cap_rows", ctypes.c_int), ("policy", ctypes.c_int)]
 
 
 class _Plan(ctypes.Structure):
@@ -93,6 +96,7 @@ class Config:
     C: float = 0.0
     gpus_per_node: int = 1
     cap_rows: int | None = None  # default S*K
+    policy: int = 0              # POLICY_ROOM or POLICY_LOCAL
 
     @property
     def cap(self) -> int:
@@ -104,7 +108,7 @@ class Config:
 
     def c(self) -> _Cfg:
         return _Cfg(self.P, self.E, self.K, self.S, self.H, self.R, float(self.C),
-                    self.gpus_per_node, self.cap)
+                    self.gpus_per_node, self.cap, self.policy)
 
 
 def validate(cfg: Config) -> int:
