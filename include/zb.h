@@ -176,8 +176,27 @@ ZB_API size_t zb_workspace_bytes(const zb_config *cfg);
 ZB_API int zb_plan(const zb_config *cfg, const int32_t *topk_ids, const zb_plan_t *plan,
             void *workspace, size_t workspace_bytes, void *stream);
 
+/* Steps 1-3 with the replica placement given instead of chosen: the slots
+ * of `placement` (device int32 [P][R], -1 = empty) are kept, and only their
+ * quotas are planned, by the same greedy restricted to existing copies (a
+ * receiver must already hold the expert; a move adds rows to that copy's
+ * quota; receivers by most room, then lowest rank).  For plans that keep a
+ * placement across invocations: Zepp "4.1 Expert Placement and Token
+ * Routing" places replicas from historical demand, and ViBE re-places only
+ * when the expert load has drifted.  `placement` may be the rep_expert of
+ * the previous plan, and may alias plan->rep_expert.  A slot naming an
+ * expert homed on its own rank, an id outside [0, E) or an expert twice on
+ * one rank makes the plan's status ZB_ERR_INVALID (reported by
+ * zb_plan_status; nothing else is written).  Other arguments, results and
+ * errors as zb_plan; rep_expert receives the placement, rep_quota the
+ * planned quotas (0 for copies that take no rows). */
+ZB_API int zb_plan_placed(const zb_config *cfg, const int32_t *topk_ids, const int32_t *placement,
+                          const zb_plan_t *plan, void *workspace, size_t workspace_bytes,
+                          void *stream);
+
 /* Synchronises `stream`, then returns the plan's status (ZB_OK,
- * ZB_WARN_UNBALANCED, ZB_ERR_CAPACITY, ZB_ERR_BAD_ID), or ZB_ERR_CUDA.
+ * ZB_WARN_UNBALANCED, ZB_ERR_CAPACITY, ZB_ERR_BAD_ID, or ZB_ERR_INVALID for
+ * a bad placement given to zb_plan_placed), or ZB_ERR_CUDA.
  * If max_load is not NULL it receives the planned max rank load (host int). */
 ZB_API int zb_plan_status(const zb_config *cfg, const zb_plan_t *plan, void *stream,
                    int32_t *max_load);

@@ -69,6 +69,8 @@ def _load():
         lib = ctypes.CDLL(build())
         lib.zbo_validate.argtypes = [ctypes.POINTER(_Cfg)]
         lib.zbo_plan.argtypes = [ctypes.POINTER(_Cfg), _P32, ctypes.POINTER(_Out)]
+        lib.zbo_plan_placed.argtypes = [ctypes.POINTER(_Cfg), _P32, _P32, ctypes.POINTER(_Out)]
+        lib.zbo_placement_valid.argtypes = [ctypes.POINTER(_Cfg), _P32]
         vp = ctypes.c_void_p
         lib.zbo_dispatch.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp]
         lib.zbo_dispatch.restype = None
@@ -116,8 +118,11 @@ def validate(cfg: Config) -> int:
     return int(_load().zbo_validate(ctypes.byref(cfg.c())))
 
 
-def plan(cfg: Config, ids: np.ndarray, want_M: bool = True) -> dict:
-    """Steps 1-3 on host arrays.  ``ids`` is int32 ``[P,S,K]``.
+def plan(cfg: Config, ids: np.ndarray, want_M: bool = True,
+         placement: np.ndarray | None = None) -> dict:
+    """Steps 1-3 on host arrays.  ``ids`` is int32 ``[P,S,K]``.  With
+    ``placement`` (int32 ``[P,R]``, -1 = empty slot) the replica placement is
+    kept and only the quotas are planned.
 
     Returns a dict with ``status`` and the plan tables (numpy int32 arrays
     shaped as the C comments state), ``M`` ``[E,P,P]`` when requested, and the
@@ -140,7 +145,11 @@ def plan(cfg: Config, ids: np.ndarray, want_M: bool = True) -> dict:
                                        "load_before", "load_after", "cu_seqlens",
                                        "dst_row", "row_src")],
                _ptr(r["M"]) if want_M else _P32(), 0, 0, 0, 0, 0)
-    st = lib.zbo_plan(ctypes.byref(cfg.c()), _ptr(ids), ctypes.byref(out))
+    if placement is None:
+        st = lib.zbo_plan(ctypes.byref(cfg.c()), _ptr(ids), ctypes.byref(out))
+    else:
+        pl = np.ascontiguousarray(placement, dtype=np.int32).reshape(P, R)
+        st = lib.zbo_plan_placed(ctypes.byref(cfg.c()), _ptr(ids), _ptr(pl), ctypes.byref(out))
     r.update(status=int(st), locality_cost=int(out.locality_cost), max_load=int(out.max_load),
              n_replicas=int(out.n_replicas), n_iters=int(out.n_iters), T=int(out.water_level))
     return r

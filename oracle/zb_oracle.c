@@ -246,6 +246,76 @@ static void greedy_place(const zbo_config *c, const int32_t *cnt, int32_t T, int
   free(nfill);
 }
 
+/* Quotas for a given replica placement (no new copies): the same greedy, but
+ * a receiver must already hold a copy of the expert, and a move adds m rows
+ * to that copy's quota.  Donor, expert and receiver order as in
+ * greedy_place with policy 0 (busiest rank, heaviest home expert, the holder
+ * with the most room, lowest ids on ties).  Each move brings the donor to T,
+ * fills the receiver to T, or exhausts the expert's home quota, so with the
+ * stuck marks there are at most 3P + E iterations.  This is the quota step
+ * of a plan that keeps its placement across invocations (Zepp 4.1, replicas
+ * placed from historical demand; ViBE, recalibration only on drift). */
+static void greedy_placed(const zbo_config *c, int32_t T, int32_t *load, int32_t *hq,
+                          const int32_t *rep_expert, int32_t *rep_quota, int32_t *n_iters) {
+  const int P = c->P, R = c->R, Eh = c->E / c->P;
+  int *stuck = calloc((size_t)P, sizeof(int));
+  int *order = malloc(sizeof(int) * (size_t)Eh);
+  for (int x = 0; x < P * R; x++) rep_quota[x] = 0;
+  *n_iters = 0;
+  for (;;) {
+    int d = -1;
+    for (int j = 0; j < P; j++)
+      if (!stuck[j] && (d < 0 || load[j] > load[d])) d = j;
+    if (d < 0 || load[d] <= T) break;
+    *n_iters += 1;
+    int n = 0;
+    for (int e = d * Eh; e < (d + 1) * Eh; e++) {
+      if (hq[e] <= 0) continue;
+      int p = n++;
+      while (p > 0 && (hq[order[p - 1]] < hq[e])) { order[p] = order[p - 1]; p--; }
+      order[p] = e;
+    }
+    int pick_e = -1, pick_r = -1, pick_s = -1;
+    for (int t = 0; t < n && pick_e < 0; t++) {
+      int e = order[t];
+      for (int r = 0; r < P; r++) {
+        if (r == d || load[r] >= T) continue;
+        for (int sl = 0; sl < R; sl++)
+          if (rep_expert[r * R + sl] == e && (pick_r < 0 || load[r] < load[pick_r])) {
+            pick_e = e;
+            pick_r = r;
+            pick_s = sl;
+          }
+      }
+    }
+    if (pick_e < 0) { stuck[d] = 1; continue; }
+    int32_t m = load[d] - T;
+    if (T - load[pick_r] < m) m = T - load[pick_r];
+    if (hq[pick_e] < m) m = hq[pick_e];
+    rep_quota[pick_r * R + pick_s] += m;
+    load[pick_r] += m;
+    load[d] -= m;
+    hq[pick_e] -= m;
+  }
+  free(order);
+  free(stuck);
+}
+
+/* A replica placement is valid when every slot is empty (-1) or names an
+ * expert homed on another rank, with no expert twice on one rank. */
+int zbo_placement_valid(const zbo_config *c, const int32_t *rep_expert) {
+  const int P = c->P, R = c->R, Eh = c->E / c->P;
+  for (int j = 0; j < P; j++)
+    for (int s = 0; s < R; s++) {
+      int e = rep_expert[j * R + s];
+      if (e == -1) continue;
+      if (e < 0 || e >= c->E || e / Eh == j) return 0;
+      for (int t = 0; t < s; t++)
+        if (rep_expert[j * R + t] == e) return 0;
+    }
+  return 1;
+}
+
 /* ------------------------- step 3: transport, groups, cu_seqlens, rows */
 
 typedef struct { int rank, group; int32_t quota; } host_t;
@@ -303,9 +373,20 @@ static int transport(const zbo_config *c, const int32_t *cnt, int e,
 /* The whole plan: steps 1-3.  Returns ZBO_OK, ZBO_UNBALANCED (some rank stays
  * above T because R slots do not permit T), or an error.  On
  * ZBO_ERR_CAPACITY the plan tables are valid but dst_row/row_src are all -1. */
+int zbo_plan_placed(const zbo_config *c, const int32_t *ids, const int32_t *placement,
+                    zbo_plan_out *out);
+
 int zbo_plan(const zbo_config *c, const int32_t *ids, zbo_plan_out *out) {
+  return zbo_plan_placed(c, ids, NULL, out);
+}
+
+/* The whole plan with the replica placement given (placement != NULL: quotas
+ * only, by greedy_placed) or chosen by the greedy (placement == NULL). */
+int zbo_plan_placed(const zbo_config *c, const int32_t *ids, const int32_t *placement,
+                    zbo_plan_out *out) {
   int rc = zbo_validate(c);
   if (rc) return rc;
+  if (placement && !zbo_placement_valid(c, placement)) return ZBO_ERR_INVALID;
   const int P = c->P, E = c->E, R = c->R, Eh = E / P, G = Eh + R;
   const int64_t NK = (int64_t)c->S * c->K;
 
@@ -329,8 +410,14 @@ int zbo_plan(const zbo_config *c, const int32_t *ids, zbo_plan_out *out) {
   out->water_level = T;
 
   for (int e = 0; e < E; e++) out->home_quota[e] = Te[e];
-  greedy_place(c, out->cnt, T, out->load_after, out->home_quota, out->rep_expert,
-               out->rep_quota, &out->n_iters);
+  if (placement) {
+    memcpy(out->rep_expert, placement, sizeof(int32_t) * (size_t)P * R);
+    greedy_placed(c, T, out->load_after, out->home_quota, out->rep_expert, out->rep_quota,
+                  &out->n_iters);
+  } else {
+    greedy_place(c, out->cnt, T, out->load_after, out->home_quota, out->rep_expert,
+                 out->rep_quota, &out->n_iters);
+  }
 
   out->max_load = 0;
   out->n_replicas = 0;

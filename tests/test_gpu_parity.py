@@ -379,3 +379,65 @@ def test_combine_special_values(dev):
     nan_w = ((want & 0x7F80) == 0x7F80) & ((want & 0x7F) != 0)
     np.testing.assert_array_equal(nan_g, nan_w)
     np.testing.assert_array_equal(got[~nan_w], want[~nan_w])
+
+
+# ------------------------------------------------------------- kept placement
+
+def _random_placement(rng, P, E, R):
+    Eh = E // P
+    pl = np.full((P, R), -1, np.int32)
+    for j in range(P):
+        others = [e for e in range(E) if e // Eh != j]
+        n = int(rng.integers(0, min(R, len(others)) + 1))
+        if n:
+            pl[j, :n] = rng.choice(others, size=n, replace=False)
+    return pl
+
+
+@pytest.mark.parametrize("k", range(0, len(SMALL), 2))
+def test_placed_random_small(dev, k):
+    """zb_plan_placed against the oracle's plan with the same placement."""
+    kw, ids = SMALL[k]
+    if kw["R"] == 0:
+        pytest.skip("no slots to place")
+    rng = np.random.default_rng(2000 + k)
+    kw = dict(kw, cap_rows=max(1, kw["P"] * kw["S"] * kw["K"]))
+    zc, oc = zb.Config(**kw), oracle.Config(**kw)
+    pl = _random_placement(rng, zc.P, zc.E, zc.R)
+    p = zb.Plan(zc, dev)
+    zb.plan_placed(p, torch.from_numpy(ids).to(dev), torch.from_numpy(pl).to(dev))
+    status, _ = zb.plan_status(p)
+    assert_plan_equal(plan_tables(p), oracle.plan(oc, ids, placement=pl), status)
+
+
+def test_placed_drift_and_aliasing(dev):
+    """The drifting workload at full size: step 0's placement kept for later
+    steps, passed as the plan's own rep_expert (aliasing is allowed)."""
+    wl = synth.WORKLOADS["drift"]
+    zc, oc = cfgs(wl, cap_rows=3 * wl.S * wl.K)
+    ids0, _ = synth.routing(wl, 0, 0)
+    p = zb.Plan(zc, dev, with_row_src=False)
+    zb.plan(p, torch.from_numpy(ids0).to(dev))
+    zb.plan_status(p)
+    o0 = oracle.plan(oc, ids0, want_M=False)
+    for step in (1, 31, 63):
+        ids, _ = synth.routing(wl, 0, step)
+        zb.plan_placed(p, torch.from_numpy(ids).to(dev), p.rep_expert)
+        status, _ = zb.plan_status(p)
+        assert_plan_equal(plan_tables(p), oracle.plan(oc, ids, want_M=False,
+                                                      placement=o0["rep_expert"]), status)
+
+
+def test_placed_invalid(dev):
+    zc = zb.Config(P=3, E=6, K=1, S=2, H=8, R=2, cap_rows=6)
+    ids = torch.zeros((3, 2, 1), dtype=torch.int32, device=dev)
+    p = zb.Plan(zc, dev)
+    for bad in ([[0, -1], [-1, -1], [-1, -1]], [[2, 2], [-1, -1], [-1, -1]],
+                [[6, -1], [-1, -1], [-1, -1]], [[-2, -1], [-1, -1], [-1, -1]]):
+        zb.plan_placed(p, ids, torch.tensor(bad, dtype=torch.int32, device=dev))
+        with pytest.raises(zb.ZbError) as err:
+            zb.plan_status(p)
+        assert err.value.status == zb.ERR_INVALID
+    zb.plan_placed(p, ids, torch.tensor([[2, 4], [0, -1], [-1, 1]], dtype=torch.int32,
+                                        device=dev))
+    assert zb.plan_status(p)[0] in (zb.OK, zb.WARN_UNBALANCED)

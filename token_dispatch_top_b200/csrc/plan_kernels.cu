@@ -227,6 +227,76 @@ __device__ void greedy_warp(const PlanArgs& a, PlannerSmem& s, int T, int load, 
   }
 }
 
+// Quotas for a given replica placement, run by one warp: the greedy of
+// greedy_warp restricted to copies that already exist (a receiver must hold
+// the expert, and the move adds to that copy's quota), receivers by most room
+// then lowest rank.  Each move brings the donor to T, fills the receiver to T
+// or exhausts the expert's home quota: at most 3P + E iterations with the
+// stuck marks.  (Zepp 4.1: replicas placed from historical demand; ViBE:
+// placement recalibrated only on drift.)
+__device__ void greedy_placed_warp(const PlanArgs& a, PlannerSmem& s, int T, int load,
+                                   int lane) {
+  const int P = a.P, R = a.R, Eh = a.Eh;
+  bool stuck = lane >= P;
+  int iters = 0;
+  const int max_iters = 3 * P + a.E + 1;
+  for (int guard = 0; guard <= max_iters; ++guard) {
+    const unsigned dl = stuck ? 0u : unsigned(load) + 1u;
+    const unsigned dmax = __reduce_max_sync(kFull, dl);
+    if (dmax == 0u) break;
+    const int d = __ffs(__ballot_sync(kFull, dl == dmax)) - 1;
+    const int dload = int(dmax - 1u);
+    if (dload <= T) break;
+    ++iters;
+    const unsigned base = __ballot_sync(kFull, lane < P && lane != d && load < T);
+    // d's heaviest home expert with a copy on some rank in base
+    unsigned bq = 0u, bx = 0xffffffffu, bh = 0u;
+    const int e0 = d * Eh;
+    for (int x = lane; x < Eh; x += 32) {
+      const unsigned q = unsigned(s.hq[e0 + x]);
+      const unsigned h = s.hold[e0 + x];
+      if (q > bq && (base & h) != 0u) {
+        bq = q;
+        bx = unsigned(x);
+        bh = h;
+      }
+    }
+    const unsigned qmax = __reduce_max_sync(kFull, bq);
+    if (qmax == 0u) {
+      if (lane == d) stuck = true;
+      continue;
+    }
+    const unsigned xmin = __reduce_min_sync(kFull, bq == qmax ? bx : 0xffffffffu);
+    const unsigned held = __shfl_sync(kFull, bh, int(xmin & 31u));
+    const int e = e0 + int(xmin);
+    const int q = int(qmax);
+    const bool elig = ((base >> lane) & 1u) && ((held >> lane) & 1u);
+    const unsigned rk = elig ? unsigned(load) : 0xffffffffu;
+    const unsigned rmin = __reduce_min_sync(kFull, rk);
+    const int r = __ffs(__ballot_sync(kFull, elig && rk == rmin)) - 1;
+    const int m = min(min(dload - T, T - int(rmin)), q);
+    if (lane == r) {
+      for (int sl = 0; sl < R; ++sl)
+        if (s.repe[r * R + sl] == e) s.repq[r * R + sl] += m;
+      load += m;
+    }
+    if (lane == d) load -= m;
+    if (lane == 0) s.hq[e] = q - m;
+    __syncwarp();
+  }
+  int nrep = 0;
+  if (lane < P)
+    for (int sl = 0; sl < R; ++sl) nrep += s.repe[lane * R + sl] >= 0;
+  if (lane < P) a.load_after[lane] = load;
+  const int mx = int(__reduce_max_sync(kFull, lane < P ? unsigned(load) : 0u));
+  nrep = int(__reduce_add_sync(kFull, unsigned(nrep)));
+  if (lane == 0) {
+    s.misc[kMiscMax] = mx;
+    s.misc[kMiscNrep] = nrep;
+    s.misc[kMiscIters] = iters;
+  }
+}
+
 // Transport of eq. (1) for expert e, run by one warp, lane = source rank.
 // Writes source lane's segments of e into the segment table and returns the
 // lane's share of the locality cost.
@@ -351,11 +421,28 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
       atomicAdd(&s.misc[kMiscBad], v);
     }
   }
+  // the replica table: empty, or the placement to keep (checked: each slot
+  // empty or an expert homed elsewhere, no expert twice on a rank)
   for (int x = tid; x < P * R; x += kPlanThreads) {
-    s.repe[x] = -1;
+    int e = -1;
+    if (a.placement) {
+      e = a.placement[x];
+      const int j = x / R, sl = x - j * R;
+      bool ok = e == -1 || (e >= 0 && e < E && e / Eh != j);
+      for (int t = 0; t < sl && ok; ++t) ok = a.placement[j * R + t] != e || e == -1;
+      if (!ok) atomicExch(&s.misc[kMiscErr], 1);
+    }
+    s.repe[x] = e;
     s.repq[x] = 0;
   }
   __syncthreads();
+  if (s.misc[kMiscErr]) {
+    if (tid == 0) {
+      for (int k = 0; k < ZB_STATS_LEN; ++k) a.stats[k] = 0;
+      a.stats[ZB_STAT_STATUS] = ZB_ERR_INVALID;
+    }
+    return;
+  }
   const int bad = s.misc[kMiscBad];
   if (bad) {
     if (tid == 0) {
@@ -365,13 +452,17 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
     }
     return;
   }
-  // T_e, the initial home quotas
+  // T_e, the initial home quotas, and the holders of each placed copy
   for (int e = tid; e < E; e += kPlanThreads) {
     int t = 0;
     for (int i = 0; i < P; ++i) t += s.cnt[i * E + e];
     s.hq[e] = t;
     s.hold[e] = 0u;
   }
+  __syncthreads();
+  if (a.placement)
+    for (int x = tid; x < P * R; x += kPlanThreads)
+      if (s.repe[x] >= 0) atomicOr(&s.hold[s.repe[x]], 1u << (x / R));
   __syncthreads();
 
   if (warp == 0) {
@@ -383,7 +474,10 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
     const long long total = warp_sum64(lane < P ? (long long)L : 0ll);
     const int T = int((total + P - 1) / P);
     if (lane == 0) s.misc[kMiscT] = T;
-    greedy_warp(a, s, T, L, lane);
+    if (a.placement)
+      greedy_placed_warp(a, s, T, L, lane);
+    else
+      greedy_warp(a, s, T, L, lane);
   }
   __syncthreads();
 

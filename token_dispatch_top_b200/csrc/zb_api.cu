@@ -65,8 +65,12 @@ size_t zb_workspace_bytes(const zb_config* c) {
   return zb::workspace_layout(*c).bytes;
 }
 
-int zb_plan(const zb_config* c, const int32_t* ids, const zb_plan_t* plan, void* ws,
-            size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+int plan_impl(const zb_config* c, const int32_t* ids, const int32_t* placement,
+              const zb_plan_t* plan, void* ws, size_t ws_bytes, void* stream) {
   if (zb_validate(c) != ZB_OK) return ZB_ERR_INVALID;
   if (!plan_buffers_ok(*c, plan)) return ZB_ERR_INVALID;
   const Workspace w = zb::workspace_layout(*c);
@@ -80,6 +84,7 @@ int zb_plan(const zb_config* c, const int32_t* ids, const zb_plan_t* plan, void*
   a.gpn = c->gpus_per_node; a.cap = c->cap_rows; a.policy = c->policy;
   a.nchunk = w.nchunk; a.seg_width = w.seg_width;
   a.ids = ids;
+  a.placement = placement;
   a.cnt = plan->cnt; a.rep_expert = plan->rep_expert; a.rep_quota = plan->rep_quota;
   a.home_quota = plan->home_quota; a.load_before = plan->load_before;
   a.load_after = plan->load_after; a.cu_seqlens = plan->cu_seqlens; a.dst_row = plan->dst_row;
@@ -96,6 +101,21 @@ int zb_plan(const zb_config* c, const int32_t* ids, const zb_plan_t* plan, void*
   if (zb::launch_planner(a, zb::planner_smem_bytes(*c), s) != cudaSuccess) return ZB_ERR_CUDA;
   if (zb::launch_assign(a, s) != cudaSuccess) return ZB_ERR_CUDA;
   return ZB_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int zb_plan(const zb_config* c, const int32_t* ids, const zb_plan_t* plan, void* ws,
+            size_t ws_bytes, void* stream) {
+  return plan_impl(c, ids, nullptr, plan, ws, ws_bytes, stream);
+}
+
+int zb_plan_placed(const zb_config* c, const int32_t* ids, const int32_t* placement,
+                   const zb_plan_t* plan, void* ws, size_t ws_bytes, void* stream) {
+  if (c && c->R > 0 && !placement) return ZB_ERR_INVALID;
+  return plan_impl(c, ids, c && c->R > 0 ? placement : nullptr, plan, ws, ws_bytes, stream);
 }
 
 int zb_plan_status(const zb_config* c, const zb_plan_t* plan, void* stream, int32_t* max_load) {

@@ -60,6 +60,7 @@ struct PlanArgs {
   int P, E, K, S, R, Eh, gpn, cap, policy;
   int nchunk, seg_width;
   const int32_t* ids;
+  const int32_t* placement;  // [P][R] replica placement to keep, or nullptr
   int32_t* cnt;
   int32_t* rep_expert;
   int32_t* rep_quota;

@@ -32,8 +32,8 @@ STAT_STATUS, STAT_MAX_LOAD, STAT_N_REPLICAS, STAT_N_ITERS, STAT_WATER_LEVEL, \
     STAT_LOCALITY_COST, STAT_BAD_IDS = range(7)
 STATS_LEN = 8
 
-EXPORTS = ("zb_strerror", "zb_validate", "zb_workspace_bytes", "zb_plan", "zb_plan_status",
-           "zb_dispatch", "zb_combine")
+EXPORTS = ("zb_strerror", "zb_validate", "zb_workspace_bytes", "zb_plan", "zb_plan_placed",
+           "zb_plan_status", "zb_dispatch", "zb_combine")
 
 
 class ZbError(RuntimeError):
@@ -73,6 +73,7 @@ def load() -> ctypes.CDLL:
         lib.zb_workspace_bytes.argtypes = [cfgp]
         lib.zb_workspace_bytes.restype = ctypes.c_size_t
         lib.zb_plan.argtypes = [cfgp, vp, planp, vp, ctypes.c_size_t, vp]
+        lib.zb_plan_placed.argtypes = [cfgp, vp, vp, planp, vp, ctypes.c_size_t, vp]
         lib.zb_plan_status.argtypes = [cfgp, planp, vp, ctypes.POINTER(ctypes.c_int32)]
         lib.zb_dispatch.argtypes = [cfgp, planp, vp, vp, vp]
         lib.zb_combine.argtypes = [cfgp, planp, vp, vp, vp, vp]
@@ -170,6 +171,20 @@ def plan(p: Plan, topk_ids: torch.Tensor, stream=None) -> None:
                         p.ws_ptr, p.ws_bytes, _stream(stream))
     if st != OK:
         raise ZbError(st, "zb_plan")
+
+
+def plan_placed(p: Plan, topk_ids: torch.Tensor, placement: torch.Tensor, stream=None) -> None:
+    """Steps 1-3 keeping a given replica placement (asynchronous).
+    ``placement``: int32 [P,R] on the device, -1 = empty slot; it may be the
+    ``rep_expert`` of this or another plan of the same shape."""
+    cfg = p.cfg
+    _check(topk_ids, (cfg.P, cfg.S, cfg.K), torch.int32, "topk_ids")
+    _check(placement, (cfg.P, cfg.R), torch.int32, "placement")
+    st = load().zb_plan_placed(ctypes.byref(p._c), topk_ids.data_ptr(),
+                               placement.data_ptr() if placement.numel() else None,
+                               ctypes.byref(p._p), p.ws_ptr, p.ws_bytes, _stream(stream))
+    if st != OK:
+        raise ZbError(st, "zb_plan_placed")
 
 
 def plan_status(p: Plan, stream=None) -> tuple[int, int]:
