@@ -16,7 +16,7 @@ step moves exactly the dispatch and combine traffic.
 * ``e2e``: the same metric through the public API with pinned host buffers:
   each step copies ids, weights and hidden rows host->device, runs the path,
   and copies the combined rows and the plan status back; the copies run on
-  their own streams with two buffer slots, so the input copy of one step
+  their own streams with three buffer slots, so the input copy of one step
   overlaps the output copy of the one before.
 * ``roofline``: the dominant kernel's algorithmic bytes per launch over its
   event-timed duration, against the measured HBM copy bandwidth.
@@ -334,13 +334,13 @@ def run_ours(args, wl, rank, world, local_rank):
     # ---- end to end through the public API, pinned host buffers.  Every step
     # copies its ids, gates and hidden rows host->device, runs plan, dispatch
     # and combine, and copies its combined rows and plan status back.  Copies
-    # run on their own streams with two buffer slots, so one step's input copy
-    # overlaps the previous step's output copy (the host link is full duplex);
-    # compute stays in order on the compute stream.
+    # run on their own streams with three buffer slots, so one step's input
+    # copy overlaps the previous step's output copy (the host link is full
+    # duplex); compute stays in order on the compute stream.
     ids_h = torch.from_numpy(ids_np).pin_memory()
     w_h = torch.from_numpy(w_np).pin_memory()
     hid_h = torch.from_numpy(hidden_np.view(np.int16)).pin_memory()
-    n_slots = 2
+    n_slots = 3
     out_h = [torch.empty((P, S, H), dtype=torch.int16).pin_memory() for _ in range(n_slots)]
     stats_h = torch.empty((max(args.steps, args.warmup), zb.STATS_LEN),
                           dtype=torch.int64).pin_memory()
@@ -436,7 +436,7 @@ def run_ours(args, wl, rank, world, local_rank):
                 "d2h_bytes_per_step": d2h,
                 "method": "pinned host buffers; per step H2D of ids, gates and hidden, "
                           "plan+dispatch+combine, D2H of out and status; copies on two "
-                          "streams with two slots (input copy of step k+1 overlaps output "
+                          "streams with three slots (input copy of step k+1 overlaps output "
                           "copy of step k); no L2 flush: each step moves 270 MB over the "
                           "host link and 1.9 GB through HBM"},
         "gpu_launches": 5 * args.steps,

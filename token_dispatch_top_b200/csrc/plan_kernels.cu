@@ -133,6 +133,7 @@ enum { kMiscT = 0, kMiscMax = 1, kMiscNrep = 2, kMiscIters = 3, kMiscBad = 4, kM
 // filled-slot count and stuck flag, and every decision is one or two warp
 // reductions.  (ISER-MoE HALO-Q Objective 1 and stages 2-3; Zepp 4.1 R slots
 // per GPU and node-first hierarchical placement.)
+template <int kPolicy>
 __device__ void greedy_warp(const PlanArgs& a, PlannerSmem& s, int T, int load, int lane) {
   const int P = a.P, R = a.R, Eh = a.Eh, gpn = a.gpn;
   int nfill = 0;
@@ -178,7 +179,7 @@ __device__ void greedy_warp(const PlanArgs& a, PlannerSmem& s, int T, int load, 
     const bool elig = ((base >> lane) & 1u) && !((hold >> lane) & 1u);
     const bool cov = ((e / Eh) / gpn == lane / gpn) || ((hold & node_mask) != 0u);
     int r, rload;
-    if (a.policy == ZB_POLICY_LOCAL) {
+    if (kPolicy == ZB_POLICY_LOCAL) {
       // balance first, locality among equal moves (HALO-Q Objective 2): after
       // node coverage, the largest move m_r, then the most own rows the copy
       // would serve locally, min(cnt[r][e], m_r), then load and rank
@@ -396,6 +397,9 @@ __device__ long long transport_warp(const PlanArgs& a, PlannerSmem& s, int e, in
   return cost;
 }
 
+// One instance per greedy mode (kMode: 0 room, 1 local, 2 kept placement), so
+// each instance carries only the greedy loop it runs.
+template <int kMode>
 __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
   extern __shared__ __align__(16) char smem_raw[];
   __shared__ unsigned long long s_cost;
@@ -425,7 +429,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
   // empty or an expert homed elsewhere, no expert twice on a rank)
   for (int x = tid; x < P * R; x += kPlanThreads) {
     int e = -1;
-    if (a.placement) {
+    if (kMode == 2) {
       e = a.placement[x];
       const int j = x / R, sl = x - j * R;
       bool ok = e == -1 || (e >= 0 && e < E && e / Eh != j);
@@ -460,7 +464,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
     s.hold[e] = 0u;
   }
   __syncthreads();
-  if (a.placement)
+  if (kMode == 2)
     for (int x = tid; x < P * R; x += kPlanThreads)
       if (s.repe[x] >= 0) atomicOr(&s.hold[s.repe[x]], 1u << (x / R));
   __syncthreads();
@@ -474,10 +478,10 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
     const long long total = warp_sum64(lane < P ? (long long)L : 0ll);
     const int T = int((total + P - 1) / P);
     if (lane == 0) s.misc[kMiscT] = T;
-    if (a.placement)
+    if (kMode == 2)
       greedy_placed_warp(a, s, T, L, lane);
     else
-      greedy_warp(a, s, T, L, lane);
+      greedy_warp<kMode>(a, s, T, L, lane);
   }
   __syncthreads();
 
@@ -658,20 +662,27 @@ cudaError_t launch_hist(const PlanArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_planner(const PlanArgs& a, size_t smem, cudaStream_t s) {
+template <int kMode>
+cudaError_t launch_planner_mode(const PlanArgs& a, size_t smem, cudaStream_t s) {
   static bool configured[64] = {};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    err = cudaFuncSetAttribute(k_planner, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    err = cudaFuncSetAttribute(k_planner<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                200 * 1024);
     if (err != cudaSuccess) return err;
     configured[dev] = true;
   }
-  k_planner<<<1, kPlanThreads, smem, s>>>(a);
+  k_planner<kMode><<<1, kPlanThreads, smem, s>>>(a);
   return cudaGetLastError();
+}
+
+cudaError_t launch_planner(const PlanArgs& a, size_t smem, cudaStream_t s) {
+  if (a.placement) return launch_planner_mode<2>(a, smem, s);
+  if (a.policy == ZB_POLICY_LOCAL) return launch_planner_mode<ZB_POLICY_LOCAL>(a, smem, s);
+  return launch_planner_mode<ZB_POLICY_ROOM>(a, smem, s);
 }
 
 cudaError_t launch_assign(const PlanArgs& a, cudaStream_t s) {
