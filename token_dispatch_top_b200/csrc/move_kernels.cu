@@ -143,7 +143,7 @@ cudaError_t dispatch_k(int ntok, int H, int64_t nrows, const int32_t* dst_row,
                        const int64_t* stats, const uint16_t* hidden, uint16_t* buf,
                        cudaStream_t s) {
   const int blocks = (ntok + kMoveWarps - 1) / kMoveWarps;
-  k_dispatch<K, 4><<<blocks, kMoveThreads, 0, s>>>(ntok, H, nrows, dst_row, stats,
+  k_dispatch<K, 8><<<blocks, kMoveThreads, 0, s>>>(ntok, H, nrows, dst_row, stats,
                                                    reinterpret_cast<const uint4*>(hidden),
                                                    reinterpret_cast<uint4*>(buf));
   return cudaGetLastError();
@@ -153,7 +153,7 @@ template <int K>
 cudaError_t combine_k(int ntok, int H, int64_t nrows, const int32_t* dst_row,
                       const int64_t* stats, const uint16_t* y, const float* w, uint16_t* out,
                       cudaStream_t s) {
-  constexpr int U = K <= 4 ? 4 : (K <= 8 ? 2 : 1);
+  constexpr int U = K <= 6 ? 4 : (K <= 8 ? 2 : 1);
   const int blocks = (ntok + kMoveWarps - 1) / kMoveWarps;
   k_combine<K, U><<<blocks, kMoveThreads, 0, s>>>(ntok, H, nrows, dst_row, stats,
                                                   reinterpret_cast<const uint4*>(y), w,
