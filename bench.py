@@ -331,6 +331,29 @@ def run_ours(args, wl, rank, world, local_rank):
     t_comb = [ev[k][2].elapsed_time(ev[k][3]) for k in range(n_ev)]
     step_ms = sum(ev[k][0].elapsed_time(ev[k][3]) for k in range(n_ev))  # total over K steps
 
+    # ---- the merged dispatch (Zepp 4.2 merge), timed apart from the step: one
+    # row per (token, destination rank) instead of one per (token, k)
+    merged = zb.Merge(cfg, dev)
+    tbuf = torch.empty_like(buf)
+    zb.plan(plan, ids)
+    zb.merge(plan, merged)
+    zb.dispatch_merged(plan, merged, hidden, tbuf)
+    torch.cuda.synchronize()
+    m_ms, d_ms = [], []
+    for _ in range(max(20, min(args.steps, 100))):
+        flush_l2()
+        a0, a1, a2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        a0.record(stream)
+        zb.merge(plan, merged)
+        a1.record(stream)
+        zb.dispatch_merged(plan, merged, hidden, tbuf)
+        a2.record(stream)
+        a2.synchronize()
+        m_ms.append(a0.elapsed_time(a1))
+        d_ms.append(a1.elapsed_time(a2))
+    rows_merged = int(merged.tok_cnt.sum())
+    del tbuf
+
     # ---- end to end through the public API, pinned host buffers.  Every step
     # copies its ids, gates and hidden rows host->device, runs plan, dispatch
     # and combine, and copies its combined rows and plan status back.  Copies
@@ -447,6 +470,13 @@ def run_ours(args, wl, rank, world, local_rank):
                        "combine": comb_ms_avg},
         "kernels_gbs": {"dispatch": ab["dispatch"] / disp_ms_avg / 1e6,
                         "combine": ab["combine"] / comb_ms_avg / 1e6},
+        "extras": {"merged_dispatch": {
+            "what": "one row per (token, destination rank), Zepp 4.2 merge; not part of the step",
+            "rows_written": rows_merged, "rows_plain": wl.N,
+            "merge_plan_ms": statistics.median(m_ms),
+            "dispatch_ms": statistics.median(d_ms),
+            "dispatch_gbs": (wl.tokens * wl.H * 2 + rows_merged * wl.H * 2 + wl.N * 4)
+            / statistics.median(d_ms) / 1e6}},
         "wall_s": wall,
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,

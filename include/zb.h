@@ -254,6 +254,45 @@ ZB_API int zb_dispatch(const zb_config *cfg, const zb_plan_t *plan, const uint16
 ZB_API int zb_combine(const zb_config *cfg, const zb_plan_t *plan, const uint16_t *y,
                const float *topk_weights, uint16_t *out, void *stream);
 
+/* ------------------------------------------------------- merged dispatch */
+
+/* The merged dispatch layout (Zepp "4.2 Split and Merge": the experts one
+ * token selects on the same destination share a single transfer).  Rank j
+ * keeps one row per token that sends it at least one entry, in (source
+ * rank, token) order, instead of one row per (token, k).  Caller-allocated
+ * device buffers (int32):
+ *   tok_row [P][S][K]  j*cap + u: the merged row of entry (i,s,k) on its
+ *                      destination rank j
+ *   grp_tok [P][cap]   for each expert-grouped row of the plan (the rows
+ *                      dst_row points at), the merged row that holds its
+ *                      data, -1 for unused rows: a grouped expert kernel
+ *                      reads grouped row p of rank j from merged row
+ *                      grp_tok[j][p]
+ *   tok_cnt [P]        rows used in rank j's merged buffer (<= load_after[j]) */
+typedef struct zb_merge_t {
+  int32_t *tok_row;
+  int32_t *grp_tok;
+  int32_t *tok_cnt;
+} zb_merge_t;
+
+/* Bytes of device scratch memory zb_merge needs (0 if cfg is invalid). */
+ZB_API size_t zb_merge_workspace_bytes(const zb_config *cfg);
+
+/* The merged layout of a completed plan (enqueued after zb_plan on the same
+ * stream).  workspace: zb_merge_workspace_bytes(cfg) bytes, 256-byte aligned.
+ * If the plan's status is an error, the buffers are left undefined.  Returns
+ * ZB_OK, ZB_ERR_INVALID or ZB_ERR_CUDA. */
+ZB_API int zb_merge(const zb_config *cfg, const zb_plan_t *plan, const zb_merge_t *merge,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/* tbuf[tok_row[i,s,k]][:] = hidden[i,s][:], each merged row written once:
+ * hidden bf16 [P][S][H] -> tbuf bf16 [P][cap][H]; rows past tok_cnt[j] are
+ * not written.  Writes a token's row once per destination rank instead of
+ * once per selected expert.  Returns ZB_OK, ZB_ERR_INVALID or ZB_ERR_CUDA. */
+ZB_API int zb_dispatch_merged(const zb_config *cfg, const zb_plan_t *plan,
+                              const zb_merge_t *merge, const uint16_t *hidden, uint16_t *tbuf,
+                              void *stream);
+
 #ifdef __cplusplus
 }
 #endif

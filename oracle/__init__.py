@@ -80,6 +80,10 @@ def _load():
         lib.zbo_f32_to_bf16.restype = ctypes.c_uint16
         lib.zbo_bf16_to_f32.argtypes = [ctypes.c_uint16]
         lib.zbo_bf16_to_f32.restype = ctypes.c_float
+        lib.zbo_merge.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, vp]
+        lib.zbo_merge.restype = None
+        lib.zbo_dispatch_merged.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp]
+        lib.zbo_dispatch_merged.restype = None
         d = ctypes.POINTER(ctypes.c_double)
         lib.zbo_metrics.argtypes = [ctypes.POINTER(_Cfg), _P32, _P32, _P32, d, d, d, d]
         lib.zbo_metrics.restype = None
@@ -184,6 +188,31 @@ def combine(cfg: Config, dst_row: np.ndarray, y_bits: np.ndarray, w: np.ndarray)
     _load().zbo_combine(ctypes.byref(cfg.c()), dst_row.ctypes.data, y_bits.ctypes.data,
                         w.ctypes.data, out.ctypes.data)
     return out
+
+
+def merge(cfg: Config, dst_row: np.ndarray) -> dict:
+    """Merged dispatch layout of a plan: ``tok_row`` [P,S,K], ``grp_tok``
+    [P,cap] and ``tok_cnt`` [P] (int32)."""
+    P, S, K = cfg.P, cfg.S, cfg.K
+    dst_row = np.ascontiguousarray(dst_row, dtype=np.int32)
+    r = dict(tok_row=np.zeros((P, S, K), np.int32), grp_tok=np.zeros((P, cfg.cap()), np.int32),
+             tok_cnt=np.zeros(P, np.int32))
+    _load().zbo_merge(ctypes.byref(cfg.c()), dst_row.ctypes.data, r["tok_row"].ctypes.data,
+                      r["grp_tok"].ctypes.data, r["tok_cnt"].ctypes.data)
+    return r
+
+
+def dispatch_merged(cfg: Config, tok_row: np.ndarray, hidden_bits: np.ndarray,
+                    tbuf_bits: np.ndarray | None = None) -> np.ndarray:
+    """Merged dispatch: one row per (token, destination rank) into ``tbuf``."""
+    P, S, H = cfg.P, cfg.S, cfg.H
+    hidden_bits = np.ascontiguousarray(hidden_bits, dtype=np.uint16).reshape(P, S, H)
+    tok_row = np.ascontiguousarray(tok_row, dtype=np.int32)
+    if tbuf_bits is None:
+        tbuf_bits = np.zeros((P, cfg.cap(), H), np.uint16)
+    _load().zbo_dispatch_merged(ctypes.byref(cfg.c()), tok_row.ctypes.data,
+                                hidden_bits.ctypes.data, tbuf_bits.ctypes.data)
+    return tbuf_bits
 
 
 def f32_to_bf16(x: float) -> int:

@@ -514,6 +514,49 @@ int zbo_plan_placed(const zbo_config *c, const int32_t *ids, const int32_t *plac
   return status;
 }
 
+/* ------------------------------------- merged dispatch (Zepp 4.2, merge) */
+
+/* One row per (token, destination rank) instead of one per (token, k): when
+ * a token's K experts include several served by the same rank, they share a
+ * single copy of its row there (Zepp, "4.2 Split and Merge": experts a token
+ * selects on the same remote node share one transfer).  Rank j's merged
+ * token buffer holds, in (source rank, token) order, the tokens that send it
+ * at least one entry.  Outputs:
+ *   tok_row [P][S][K]  j*cap + u: the merged row of entry (i,s,k), j its rank
+ *   grp_tok [P][cap]   for each expert-grouped row (the rows dst_row points
+ *                      at), the merged row that holds its data; -1 if unused
+ *   tok_cnt [P]        tokens merged into rank j
+ * The expert-grouped rows of the plain dispatch are then grp_tok-gathers of
+ * the merged buffer.  dst_row must be a valid plan's (all rows assigned). */
+void zbo_merge(const zbo_config *c, const int32_t *dst_row, int32_t *tok_row, int32_t *grp_tok,
+               int32_t *tok_cnt) {
+  const int P = c->P, K = c->K;
+  const int64_t cap = c->cap_rows;
+  for (int j = 0; j < P; j++) tok_cnt[j] = 0;
+  for (int64_t x = 0; x < (int64_t)P * cap; x++) grp_tok[x] = -1;
+  for (int64_t t = 0; t < (int64_t)P * c->S; t++) {
+    int32_t row_of_rank[32];
+    for (int j = 0; j < P; j++) row_of_rank[j] = -1;
+    for (int k = 0; k < K; k++) {
+      int32_t d = dst_row[t * K + k];
+      int j = (int)(d / cap);
+      if (row_of_rank[j] < 0) row_of_rank[j] = (int32_t)(j * cap + tok_cnt[j]++);
+      tok_row[t * K + k] = row_of_rank[j];
+      grp_tok[d] = row_of_rank[j];
+    }
+  }
+}
+
+/* tbuf[tok_row[i,s,k]] = hidden[i,s]: each merged row written once. */
+void zbo_dispatch_merged(const zbo_config *c, const int32_t *tok_row, const uint16_t *hidden,
+                         uint16_t *tbuf) {
+  const int64_t H = c->H;
+  for (int64_t t = 0; t < (int64_t)c->P * c->S; t++)
+    for (int k = 0; k < c->K; k++)
+      memcpy(tbuf + (int64_t)tok_row[t * c->K + k] * H, hidden + t * H,
+             sizeof(uint16_t) * (size_t)H);
+}
+
 /* ------------------------------------------------ bf16 (IEEE definition) */
 
 /* bf16 is the upper half of an IEEE binary32: widening is exact. */

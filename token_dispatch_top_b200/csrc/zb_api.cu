@@ -140,6 +140,48 @@ int zb_dispatch(const zb_config* c, const zb_plan_t* plan, const uint16_t* hidde
   return ZB_OK;
 }
 
+size_t zb_merge_workspace_bytes(const zb_config* c) {
+  if (zb_validate(c) != ZB_OK) return 0;
+  const int64_t nchunk = zb::ceil_div(int64_t(c->P) * c->S, zb::kMergeChunk);
+  return zb::align256(size_t(sizeof(int32_t)) * size_t(nchunk) * c->P + 1);
+}
+
+int zb_merge(const zb_config* c, const zb_plan_t* plan, const zb_merge_t* m, void* ws,
+             size_t ws_bytes, void* stream) {
+  if (zb_validate(c) != ZB_OK || !plan || !plan->stats || !m) return ZB_ERR_INVALID;
+  if (!m->tok_cnt || !m->grp_tok) return ZB_ERR_INVALID;
+  if (c->S > 0 && (!plan->dst_row || !m->tok_row)) return ZB_ERR_INVALID;
+  if (!ws || ws_bytes < zb_merge_workspace_bytes(c) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return ZB_ERR_INVALID;
+  if (!plan->load_after) return ZB_ERR_INVALID;
+  cudaStream_t s = as_stream(stream);
+  zb::MergeArgs a{};
+  a.P = c->P; a.K = c->K; a.cap = c->cap_rows; a.ntok = int64_t(c->P) * c->S;
+  if (a.ntok == 0) {  // no tokens: no kernel runs, every row is unused
+    if (cudaMemsetAsync(m->grp_tok, 0xff, sizeof(int32_t) * size_t(c->P) * c->cap_rows, s) !=
+            cudaSuccess ||
+        cudaMemsetAsync(m->tok_cnt, 0, sizeof(int32_t) * size_t(c->P), s) != cudaSuccess)
+      return ZB_ERR_CUDA;
+    return ZB_OK;
+  }
+  a.dst_row = plan->dst_row; a.load_after = plan->load_after; a.stats = plan->stats;
+  a.tok_row = m->tok_row; a.grp_tok = m->grp_tok; a.tok_cnt = m->tok_cnt;
+  a.chunk_cnt = static_cast<int32_t*>(ws);
+  if (zb::launch_merge(a, s) != cudaSuccess) return ZB_ERR_CUDA;
+  return ZB_OK;
+}
+
+int zb_dispatch_merged(const zb_config* c, const zb_plan_t* plan, const zb_merge_t* m,
+                       const uint16_t* hidden, uint16_t* tbuf, void* stream) {
+  if (zb_validate(c) != ZB_OK || !plan || !plan->stats || !m) return ZB_ERR_INVALID;
+  if (c->S > 0 && (!m->tok_row || !hidden || !tbuf)) return ZB_ERR_INVALID;
+  if ((hidden && !aligned16(hidden)) || (tbuf && !aligned16(tbuf))) return ZB_ERR_INVALID;
+  if (zb::launch_dispatch_merged(c->P, c->S, c->K, c->H, c->cap_rows, m->tok_row, plan->stats,
+                                 hidden, tbuf, as_stream(stream)) != cudaSuccess)
+    return ZB_ERR_CUDA;
+  return ZB_OK;
+}
+
 int zb_combine(const zb_config* c, const zb_plan_t* plan, const uint16_t* y, const float* w,
                uint16_t* out, void* stream) {
   if (zb_validate(c) != ZB_OK || !plan || !plan->stats) return ZB_ERR_INVALID;

@@ -76,6 +76,21 @@ struct PlanArgs {
   int2* seg;
 };
 
+// Tokens per CTA of the merged-dispatch layout kernels.
+constexpr int kMergeChunk = 256;
+
+struct MergeArgs {
+  int P, K, cap;
+  int64_t ntok;
+  const int32_t* dst_row;
+  const int32_t* load_after;
+  const int64_t* stats;
+  int32_t* tok_row;
+  int32_t* grp_tok;
+  int32_t* tok_cnt;
+  int32_t* chunk_cnt;  // workspace [nchunk][P]
+};
+
 size_t planner_smem_bytes(const zb_config& c);
 
 cudaError_t launch_hist(const PlanArgs& a, cudaStream_t s);
@@ -85,6 +100,10 @@ cudaError_t launch_assign(const PlanArgs& a, cudaStream_t s);
 cudaError_t launch_dispatch(int P, int S, int K, int H, int cap, const int32_t* dst_row,
                             const int64_t* stats, const uint16_t* hidden, uint16_t* buf,
                             cudaStream_t s);
+cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s);
+cudaError_t launch_dispatch_merged(int P, int S, int K, int H, int cap, const int32_t* tok_row,
+                                   const int64_t* stats, const uint16_t* hidden, uint16_t* tbuf,
+                                   cudaStream_t s);
 cudaError_t launch_combine(int P, int S, int K, int H, int cap, const int32_t* dst_row,
                            const int64_t* stats, const uint16_t* y, const float* w,
                            uint16_t* out, cudaStream_t s);

@@ -33,7 +33,8 @@ STAT_STATUS, STAT_MAX_LOAD, STAT_N_REPLICAS, STAT_N_ITERS, STAT_WATER_LEVEL, \
 STATS_LEN = 8
 
 EXPORTS = ("zb_strerror", "zb_validate", "zb_workspace_bytes", "zb_plan", "zb_plan_placed",
-           "zb_plan_status", "zb_dispatch", "zb_combine")
+           "zb_plan_status", "zb_dispatch", "zb_combine", "zb_merge_workspace_bytes",
+           "zb_merge", "zb_dispatch_merged")
 
 
 class ZbError(RuntimeError):
@@ -53,6 +54,10 @@ class _Plan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("cnt", "rep_expert", "rep_quota", "home_quota", "load_before", "load_after",
                  "cu_seqlens", "dst_row", "row_src", "stats")]
+
+
+class _Merge(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("tok_row", "grp_tok", "tok_cnt")]
 
 
 _lib = None
@@ -77,6 +82,11 @@ def load() -> ctypes.CDLL:
         lib.zb_plan_status.argtypes = [cfgp, planp, vp, ctypes.POINTER(ctypes.c_int32)]
         lib.zb_dispatch.argtypes = [cfgp, planp, vp, vp, vp]
         lib.zb_combine.argtypes = [cfgp, planp, vp, vp, vp, vp]
+        mergep = ctypes.POINTER(_Merge)
+        lib.zb_merge_workspace_bytes.argtypes = [cfgp]
+        lib.zb_merge_workspace_bytes.restype = ctypes.c_size_t
+        lib.zb_merge.argtypes = [cfgp, planp, mergep, vp, ctypes.c_size_t, vp]
+        lib.zb_dispatch_merged.argtypes = [cfgp, planp, mergep, vp, vp, vp]
         _lib = lib
     return _lib
 
@@ -220,3 +230,42 @@ def combine(p: Plan, y: torch.Tensor, topk_weights: torch.Tensor, out: torch.Ten
                            topk_weights.data_ptr(), out.data_ptr(), _stream(stream))
     if st != OK:
         raise ZbError(st, "zb_combine")
+
+
+class Merge:
+    """Device buffers of the merged dispatch layout of one plan shape."""
+
+    def __init__(self, cfg: Config, device):
+        i32 = dict(dtype=torch.int32, device=device)
+        self.cfg = cfg
+        self.tok_row = torch.empty((cfg.P, cfg.S, cfg.K), **i32)
+        self.grp_tok = torch.empty((cfg.P, cfg.cap), **i32)
+        self.tok_cnt = torch.empty((cfg.P,), **i32)
+        self.ws_bytes = int(load().zb_merge_workspace_bytes(ctypes.byref(cfg.c())))
+        self.workspace = torch.empty((self.ws_bytes + 256,), dtype=torch.uint8, device=device)
+        self.ws_ptr = (self.workspace.data_ptr() + 255) & ~255
+
+        def p(t):
+            return None if t.numel() == 0 else t.data_ptr()
+        self._m = _Merge(p(self.tok_row), p(self.grp_tok), p(self.tok_cnt))
+
+
+def merge(p: Plan, m: Merge, stream=None) -> None:
+    """The merged layout of plan ``p`` (asynchronous, after zb.plan)."""
+    st = load().zb_merge(ctypes.byref(p._c), ctypes.byref(p._p), ctypes.byref(m._m), m.ws_ptr,
+                         m.ws_bytes, _stream(stream))
+    if st != OK:
+        raise ZbError(st, "zb_merge")
+
+
+def dispatch_merged(p: Plan, m: Merge, hidden: torch.Tensor, tbuf: torch.Tensor,
+                    stream=None) -> None:
+    """One row per (token, destination rank): ``hidden`` bf16 [P,S,H] ->
+    ``tbuf`` bf16 [P,cap,H] (rows past m.tok_cnt untouched)."""
+    cfg = p.cfg
+    _check(hidden, (cfg.P, cfg.S, cfg.H), torch.bfloat16, "hidden")
+    _check(tbuf, (cfg.P, cfg.cap, cfg.H), torch.bfloat16, "tbuf")
+    st = load().zb_dispatch_merged(ctypes.byref(p._c), ctypes.byref(p._p), ctypes.byref(m._m),
+                                   hidden.data_ptr(), tbuf.data_ptr(), _stream(stream))
+    if st != OK:
+        raise ZbError(st, "zb_dispatch_merged")
