@@ -45,7 +45,8 @@ class _Cfg(ctypes.Structure):
     _fields_ = [("P", ctypes.c_int), ("E", ctypes.c_int), ("K", ctypes.c_int),
                 ("S", ctypes.c_int), ("H", ctypes.c_int), ("R", ctypes.c_int),
                 ("C", ctypes.c_double), ("gpus_per_node", ctypes.c_int),
-                ("cap_rows", ctypes.c_int), ("policy", ctypes.c_int)]
+                ("cap_rows", ctypes.c_int), ("policy", ctypes.c_int),
+                ("relax", ctypes.c_int)]
 
 
 _P32 = ctypes.POINTER(ctypes.c_int32)
@@ -93,7 +94,8 @@ def _load():
 
 @dataclass
 class Config:
-    """Problem shape.  ``cap_rows`` defaults to S*K (the water level)."""
+    """Problem shape.  ``cap_rows`` defaults to S*K (the water level), or with
+    ``relax`` to floor((1+C) S*K), C taken to 20 fractional bits (eq. (1))."""
     P: int
     E: int
     K: int
@@ -104,13 +106,20 @@ class Config:
     gpus_per_node: int = 1
     cap_rows: int | None = None
     policy: int = 0  # receiver choice: 0 most room, 1 most local rows
+    relax: int = 0   # 1: hosts receive within q +- floor(C q) (eq. (1))
 
     def cap(self) -> int:
-        return self.S * self.K if self.cap_rows is None else self.cap_rows
+        if self.cap_rows is not None:
+            return self.cap_rows
+        sk = self.S * self.K
+        if not self.relax:
+            return sk
+        cfix = int(np.floor(float(np.float32(self.C)) * 1048576.0))
+        return sk + ((sk * cfix) >> 20)
 
     def c(self) -> _Cfg:
         return _Cfg(self.P, self.E, self.K, self.S, self.H, self.R, float(self.C),
-                    self.gpus_per_node, self.cap(), self.policy)
+                    self.gpus_per_node, self.cap(), self.policy, self.relax)
 
 
 def _ptr(a: np.ndarray):

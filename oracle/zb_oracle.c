@@ -35,8 +35,11 @@
  *    routings): after node coverage, the largest move m_r = min(load_d - T,
  *    T - load_r, quota_e), then the most rows of the receiver's own demand
  *    the copy would serve, min(cnt[r][e], m_r), then lowest load and rank.
- *  - quotas are delivered exactly (|sum_i M_ij - q_j| = 0 <= C*q_j), because
- *    T = S*K leaves no slack in the fixed S*K buffers.
+ *  - by default quotas are delivered exactly (|sum_i M_ij - q_j| = 0 <=
+ *    C*q_j), because T = S*K leaves no slack in fixed S*K buffers.  With
+ *    relax = 1 each host of quota q receives between q - dl and q + dl rows,
+ *    dl = floor(q * C) with C taken to 20 fractional bits, and the receive
+ *    buffers hold floor((1+C) T) rows [ZEPP 4.1, eq. (1)]; see transport().
  *  - rows inside a group are ordered by (source rank, flat index s*K+k).
  *  - combine: acc = +0.0f; acc = fmaf(w_k, y_k, acc) for k = 0..K-1; the
  *    result is rounded to bf16 to nearest, ties to even.
@@ -63,10 +66,11 @@ typedef struct {
   int S;             /* tokens per rank */
   int H;             /* hidden width (bf16 elements per row) */
   int R;             /* replica (helper) slots per rank */
-  double C;          /* relaxation ratio of eq. (1); validated, recorded */
+  double C;          /* relaxation ratio of eq. (1); used when relax = 1 */
   int gpus_per_node; /* 1 = flat locality cost; >1 = two-level cost */
   int cap_rows;      /* rows of each rank's receive buffer (>= S*K) */
   int policy;        /* receiver choice: 0 most room, 1 most local rows */
+  int relax;         /* 0 quotas met exactly; 1 within the band of eq. (1) */
 } zbo_config;
 
 typedef struct {
@@ -115,6 +119,7 @@ int zbo_validate(const zbo_config *c) {
   if ((int64_t)c->P * c->S * c->K > INT32_MAX) return ZBO_ERR_INVALID;
   if ((int64_t)c->P * c->cap_rows > INT32_MAX) return ZBO_ERR_INVALID;
   if (c->policy != 0 && c->policy != 1) return ZBO_ERR_INVALID;
+  if (c->relax != 0 && c->relax != 1) return ZBO_ERR_INVALID;
   return ZBO_OK;
 }
 
@@ -338,35 +343,76 @@ static int hosts_of(const zbo_config *c, int e, const int32_t *home_quota,
   return n;
 }
 
+/* C as a multiple of 2^-20: floor(float(C) * 2^20).  The band half-width of a
+ * host with quota q is then floor(q * cfix / 2^20) <= C q, an integer both
+ * sides of a check compute identically.  0 when relax is off. */
+static int64_t band_cfix(const zbo_config *c) {
+  if (!c->relax) return 0;
+  return (int64_t)floor((double)(float)c->C * 1048576.0);
+}
+static int32_t band_half(int32_t q, int64_t cfix) { return (int32_t)(((int64_t)q * cfix) >> 20); }
+
 /* Locality-preferred routing, eq. (1) [ZEPP 4.1] with the local-first route
- * rewrite [ISER, HALO-Q stage 5]: serve each host's quota from the host's own
- * rank first (a=0), then for every cost level in increasing order, hosts in
- * ascending rank, sources in ascending rank.  Writes M[i*P+j] for expert e. */
+ * rewrite [ISER, HALO-Q stage 5].  Host h of quota q_h may receive between
+ * lo_h = q_h - dl_h and hi_h = q_h + dl_h rows (dl_h = 0 unless relaxed), and
+ * every row of the expert is received somewhere.  The slack D - sum lo_h
+ * (D = sum q_h, the expert's demand) is how many rows may go above the lower
+ * bounds in total; spending it never leaves a lower bound unmet.
+ *  1. each host serves its own rank (a = 0) up to lo_h;
+ *  2. hosts in ascending rank serve more of their own rank, up to hi_h, while
+ *     slack lasts;
+ *  3. for each cost level in increasing order, hosts in ascending rank take
+ *     from sources in ascending rank: first up to lo_h, then up to hi_h while
+ *     slack lasts.
+ * Step 1-2 maximise the locally served rows; with the flat cost that is the
+ * optimum of eq. (1).  Exact quotas are the case dl = 0.
+ * Writes M[i*P+j] for expert e. */
 static int transport(const zbo_config *c, const int32_t *cnt, int e,
-                     const host_t *hosts, int nh, int32_t *M) {
+                     const host_t *hosts, int nh, int64_t cfix, int32_t *M) {
   const int P = c->P;
-  int32_t dres[32], qres[33];
+  int32_t dres[32], lo[33], hi[33], recv[33];
+  int64_t slack = 0;
   memset(M, 0, sizeof(int32_t) * (size_t)P * P);
   for (int i = 0; i < P; i++) dres[i] = cnt[(size_t)i * c->E + e];
-  for (int h = 0; h < nh; h++) qres[h] = hosts[h].quota;
   for (int h = 0; h < nh; h++) {
+    int32_t dl = band_half(hosts[h].quota, cfix);
+    lo[h] = hosts[h].quota - dl;
+    hi[h] = hosts[h].quota + dl;
+    recv[h] = 0;
+    slack += dl; /* sum_h q_h - sum_h lo_h */
+  }
+  for (int h = 0; h < nh; h++) { /* 1: own rank, up to the lower bound */
     int j = hosts[h].rank;
-    int32_t take = dres[j] < qres[h] ? dres[j] : qres[h];
-    M[j * P + j] += take; dres[j] -= take; qres[h] -= take;
+    int32_t take = dres[j] < lo[h] ? dres[j] : lo[h];
+    M[j * P + j] += take; dres[j] -= take; recv[h] += take;
+  }
+  for (int h = 0; h < nh; h++) { /* 2: own rank, into the band */
+    int j = hosts[h].rank;
+    int64_t take = dres[j];
+    if (hi[h] - recv[h] < take) take = hi[h] - recv[h];
+    if (slack < take) take = slack;
+    if (take <= 0) continue;
+    M[j * P + j] += (int32_t)take; dres[j] -= (int32_t)take; recv[h] += (int32_t)take;
+    slack -= take;
   }
   int levels[2] = {1, 4};
   int nlev = c->gpus_per_node > 1 ? 2 : 1;
-  for (int l = 0; l < nlev; l++)
+  for (int l = 0; l < nlev; l++) /* 3: the other ranks, by cost level */
     for (int h = 0; h < nh; h++) {
       int j = hosts[h].rank;
       for (int i = 0; i < P; i++) {
         if (cost_a(c, i, j) != levels[l]) continue;
-        int32_t take = dres[i] < qres[h] ? dres[i] : qres[h];
-        M[i * P + j] += take; dres[i] -= take; qres[h] -= take;
+        int64_t need = recv[h] < lo[h] ? lo[h] - recv[h] : 0;
+        int64_t room = hi[h] - (recv[h] > lo[h] ? recv[h] : lo[h]);
+        if (room > slack) room = slack;
+        int64_t take = dres[i] < need + room ? dres[i] : need + room;
+        M[i * P + j] += (int32_t)take; dres[i] -= (int32_t)take; recv[h] += (int32_t)take;
+        if (take > need) slack -= take - need;
       }
     }
   for (int i = 0; i < P; i++) if (dres[i] != 0) return ZBO_ERR_INTERNAL;
-  for (int h = 0; h < nh; h++) if (qres[h] != 0) return ZBO_ERR_INTERNAL;
+  for (int h = 0; h < nh; h++)
+    if (recv[h] < lo[h] || recv[h] > hi[h]) return ZBO_ERR_INTERNAL;
   return ZBO_OK;
 }
 
@@ -426,12 +472,13 @@ int zbo_plan_placed(const zbo_config *c, const int32_t *ids, const int32_t *plac
   for (int x = 0; x < P * R; x++) out->n_replicas += out->rep_expert[x] >= 0;
 
   /* Transport per expert, kept whole: Mall[e][i][j]. */
+  const int64_t cfix = band_cfix(c);
   int32_t *Mall = calloc((size_t)E * P * P, sizeof(int32_t));
   host_t hosts[33];
   out->locality_cost = 0;
   for (int e = 0; e < E; e++) {
     int nh = hosts_of(c, e, out->home_quota, out->rep_expert, out->rep_quota, hosts);
-    rc = transport(c, out->cnt, e, hosts, nh, Mall + (size_t)e * P * P);
+    rc = transport(c, out->cnt, e, hosts, nh, cfix, Mall + (size_t)e * P * P);
     if (rc) { free(Mall); free(Te); return rc; }
     for (int i = 0; i < P; i++)
       for (int j = 0; j < P; j++)
@@ -454,7 +501,14 @@ int zbo_plan_placed(const zbo_config *c, const int32_t *ids, const int32_t *plac
     }
   }
 
+  /* Objective 1 is judged on the quota loads; the buffers must hold the rows
+   * each rank receives, its quota load or (relaxed) a load within the band. */
   int status = out->max_load > T ? ZBO_UNBALANCED : ZBO_OK;
+  out->max_load = 0;
+  for (int j = 0; j < P; j++) {
+    out->load_after[j] = out->cu_seqlens[(size_t)j * (G + 1) + G];
+    if (out->load_after[j] > out->max_load) out->max_load = out->load_after[j];
+  }
   const int64_t cap = c->cap_rows;
   if (out->row_src)
     for (int64_t x = 0; x < (int64_t)P * cap; x++) out->row_src[x] = -1;

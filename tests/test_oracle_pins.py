@@ -21,7 +21,8 @@ GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_examples.json")
 def _cfg(d):
     return oracle.Config(P=d["P"], E=d["E"], K=d["K"], S=d["S"], H=d["H"], R=d["R"],
                          C=d.get("C", 0.0), gpus_per_node=d.get("gpus_per_node", 1),
-                         cap_rows=d.get("cap_rows"), policy=d.get("policy", 0))
+                         cap_rows=d.get("cap_rows"), policy=d.get("policy", 0),
+                         relax=d.get("relax", 0))
 
 
 def _examples():
@@ -48,6 +49,11 @@ def test_hand_examples(ex):
     for key in ("r_imb_before", "r_imb_after", "maxvio", "excess_removed"):
         if key in exp:
             assert m[key] == pytest.approx(exp[key], abs=1e-12)
+    if "cap" in exp:
+        assert cfg.cap() == exp["cap"]
+    if "locality_cost_exact_quotas" in exp:
+        cfg0 = _cfg(dict(ex["cfg"], relax=0))
+        assert oracle.plan(cfg0, ids)["locality_cost"] == exp["locality_cost_exact_quotas"]
     if "status_with_cap_rows_3" in exp:
         cfg.cap_rows = 3
         assert oracle.plan(cfg, ids)["status"] == exp["status_with_cap_rows_3"]
