@@ -32,6 +32,7 @@ time.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -354,6 +355,32 @@ def run_ours(args, wl, rank, world, local_rank):
     rows_merged = int(merged.tok_cnt.sum())
     del tbuf
 
+    # ---- the banded plan (eq. (1) with its C band in use), timed apart from
+    # the step: the same ids planned with relax = 1 and floor((1+C) S*K) rows
+    cfg_b = dataclasses.replace(cfg, relax=1, cap_rows=None)
+    plan_b = zb.Plan(cfg_b, dev, with_row_src=False)
+    zb.plan(plan_b, ids)
+    torch.cuda.synchronize()
+    b_ms = []
+    for _ in range(max(20, min(args.steps, 100))):
+        flush_l2()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        zb.plan(plan_b, ids)
+        a1.record(stream)
+        a1.synchronize()
+        b_ms.append(a0.elapsed_time(a1))
+    st_b = plan_b.stats.cpu().numpy()
+    st_x = plan.stats.cpu().numpy()
+    banded = {
+        "what": f"plan with relax = 1, C = {cfg.C}: hosts receive q +- floor(C q) rows "
+                "(Zepp 4.1 eq. (1)); not part of the step",
+        "status": int(st_b[zb.STAT_STATUS]), "plan_ms": statistics.median(b_ms),
+        "cap_rows": cfg_b.cap, "max_load": int(st_b[zb.STAT_MAX_LOAD]),
+        "locality_cost": int(st_b[zb.STAT_LOCALITY_COST]),
+        "locality_cost_exact": int(st_x[zb.STAT_LOCALITY_COST])}
+    del plan_b
+
     # ---- end to end through the public API, pinned host buffers.  Every step
     # copies its ids, gates and hidden rows host->device, runs plan, dispatch
     # and combine, and copies its combined rows and plan status back.  Copies
@@ -476,7 +503,8 @@ def run_ours(args, wl, rank, world, local_rank):
             "merge_plan_ms": statistics.median(m_ms),
             "dispatch_ms": statistics.median(d_ms),
             "dispatch_gbs": (wl.tokens * wl.H * 2 + rows_merged * wl.H * 2 + wl.N * 4)
-            / statistics.median(d_ms) / 1e6}},
+            / statistics.median(d_ms) / 1e6},
+            "banded_plan": banded},
         "wall_s": wall,
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,

@@ -60,8 +60,9 @@ extern "C" {
  *   K   top-K, 1..16          S  tokens per rank, >= 0
  *   H   hidden width in bf16 elements, H >= 8, H % 8 == 0
  *   R   replica (helper) slots per rank, 0..P-1
- *   C   relaxation ratio of the routing constraint |sum_i M_ij - q_j| <= C q_j,
- *       0 <= C < 1 (validated and recorded; quotas are met exactly, see zb_plan)
+ *   C   relaxation ratio of the routing constraint |sum_i M_ij - q_j| <= C q_j
+ *       of eq. (1) (Zepp, 4.1 Expert Placement and Token Routing), 0 <= C < 1;
+ *       used only when relax = 1
  *   gpus_per_node  1 = flat locality cost; g > 1 groups ranks into nodes of g
  *       consecutive ranks (P % g == 0)
  *   cap_rows  rows of each rank's receive buffer, >= S*K; P*cap_rows and
@@ -75,7 +76,16 @@ extern "C" {
  *         expert the copy would serve locally are most, min(cnt[r][e], m_r),
  *         then the lowest load, then the lowest rank (ISER-MoE, HALO-Q
  *         Objective 2: the most locally computed tokens among balanced
- *         routings). */
+ *         routings).
+ *   relax   0: every host of an expert receives exactly its quota q (the
+ *         default; fixed S*K buffers leave no slack).  1: each host receives
+ *         between q - dl and q + dl rows, dl = floor(q * floor(C * 2^20) / 2^20),
+ *         so more rows are served on their own rank: own-rank rows up to
+ *         q - dl, then more own-rank rows in ascending host rank while the band's
+ *         total slack (sum of dl) lasts, then the other ranks by cost level.
+ *         When the quota loads reach T, a rank receives at most
+ *         T + floor(T * floor(C * 2^20) / 2^20) = floor((1+C) T) rows; size
+ *         cap_rows for that (a plan needing more is ZB_ERR_CAPACITY). */
 #define ZB_POLICY_ROOM 0
 #define ZB_POLICY_LOCAL 1
 typedef struct zb_config {
@@ -84,6 +94,7 @@ typedef struct zb_config {
   int gpus_per_node;
   int cap_rows;
   int policy;
+  int relax;
 } zb_config;
 
 /* Indices into plan->stats (int64). */
@@ -103,7 +114,8 @@ typedef struct zb_config {
  *   rep_quota   [P][R]        rows that slot receives (0 if empty)
  *   home_quota  [E]           rows the home copy of e receives
  *   load_before [P]           L_j = rows homed on j before planning
- *   load_after  [P]           rows rank j receives after planning
+ *   load_after  [P]           rows rank j receives after planning (its
+ *                             quota load; with relax, within the band)
  *   cu_seqlens  [P][Eh+R+1]   exclusive prefix of the rows of rank j's groups:
  *                             groups 0..Eh-1 are its home experts j*Eh+g,
  *                             groups Eh..Eh+R-1 its helper slots 0..R-1

@@ -13,9 +13,9 @@ PLAN_KEYS = ("cnt", "rep_expert", "rep_quota", "home_quota", "load_before", "loa
 SENTINEL = 0x7E11  # bf16 bit pattern marking rows nobody may write
 
 
-def cfgs(wl: synth.Workload, cap_rows=None, policy=0):
-    kw = dict(P=wl.P, E=wl.E, K=wl.K, S=wl.S, H=wl.H, R=wl.R, C=wl.C,
-              gpus_per_node=wl.gpus_per_node, cap_rows=cap_rows, policy=policy)
+def cfgs(wl: synth.Workload, cap_rows=None, policy=0, relax=0, C=None):
+    kw = dict(P=wl.P, E=wl.E, K=wl.K, S=wl.S, H=wl.H, R=wl.R, C=wl.C if C is None else C,
+              gpus_per_node=wl.gpus_per_node, cap_rows=cap_rows, policy=policy, relax=relax)
     return zb.Config(**kw), oracle.Config(**kw)
 
 

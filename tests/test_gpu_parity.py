@@ -76,9 +76,9 @@ def full_parity(zc, oc, ids, w, hidden_bits, y_bits, dev, with_row_src=True, str
 @pytest.mark.parametrize("ex", json.load(open(GOLDEN))["examples"], ids=lambda e: e["name"])
 def test_hand_examples(dev, ex):
     d = ex["cfg"]
-    kw = dict(P=d["P"], E=d["E"], K=d["K"], S=d["S"], H=d["H"], R=d["R"],
+    kw = dict(P=d["P"], E=d["E"], K=d["K"], S=d["S"], H=d["H"], R=d["R"], C=d.get("C", 0.0),
               gpus_per_node=d.get("gpus_per_node", 1), cap_rows=d.get("cap_rows"),
-              policy=d.get("policy", 0))
+              policy=d.get("policy", 0), relax=d.get("relax", 0))
     zc, oc = zb.Config(**kw), oracle.Config(**kw)
     ids = np.array(ex["ids"], np.int32).reshape(zc.P, zc.S, zc.K)
     rng = np.random.default_rng(0)

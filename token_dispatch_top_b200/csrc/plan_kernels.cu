@@ -127,7 +127,10 @@ __device__ PlannerSmem carve(char* base, const PlanArgs& a) {
   return s;
 }
 
-enum { kMiscT = 0, kMiscMax = 1, kMiscNrep = 2, kMiscIters = 3, kMiscBad = 4, kMiscErr = 5 };
+enum {
+  kMiscT = 0, kMiscMax = 1, kMiscNrep = 2, kMiscIters = 3, kMiscBad = 4, kMiscErr = 5,
+  kMiscRecv = 6  // banded plans: the most rows any rank receives
+};
 
 // Greedy replica placement, run by one warp; lane r holds rank r's load,
 // filled-slot count and stuck flag, and every decision is one or two warp
@@ -298,38 +301,36 @@ __device__ void greedy_placed_warp(const PlanArgs& a, PlannerSmem& s, int T, int
   }
 }
 
-// Transport of eq. (1) for expert e, run by one warp, lane = source rank.
-// Writes source lane's segments of e into the segment table and returns the
-// lane's share of the locality cost.
-__device__ long long transport_warp(const PlanArgs& a, PlannerSmem& s, int e, int lane,
-                                    int32_t* Mw, int32_t* qw) {
-  const int P = a.P, R = a.R, Eh = a.Eh, G = Eh + R, gpn = a.gpn;
-  const int h0 = e / Eh;
-  const unsigned hold = s.hold[e];
-  const int d = lane < P ? s.cnt[lane * a.E + e] : 0;
-  int2* seg = a.seg + int64_t(lane) * a.seg_width + s.hoff[e];
-  if (hold == 0u) {
-    // the home rank is the only host: every source sends it all its rows
-    const int inc = warp_incl_scan(d, lane);
-    if (lane < P)
-      seg[0] = make_int2(d, h0 * a.cap + s.cu[h0 * (G + 1) + (e - h0 * Eh)] + inc - d);
-    return (long long)cost_a(lane, h0, gpn) * d;
+// Host j's quota for expert e and the group that receives it on j.
+__device__ __forceinline__ void host_quota(const PlanArgs& a, const PlannerSmem& s, int e,
+                                           int h0, int j, int& q, int& grp) {
+  if (j == h0) {
+    q = s.hq[e];
+    grp = e - h0 * a.Eh;
+    return;
   }
-  const unsigned hostmask = hold | (1u << h0);
-  const int nh = __popc(hostmask);
-  int dres = d;
-  for (int t = 0; t < nh; ++t) Mw[t * 32 + lane] = 0;
-  __syncwarp();
-  if (lane < P && ((hostmask >> lane) & 1u)) {
-    int q = 0;
-    if (lane == h0) {
-      q = s.hq[e];
-    } else {
-      for (int r = 0; r < R; ++r)
-        if (s.repe[lane * R + r] == e) q = s.repq[lane * R + r];
+  q = 0;
+  grp = a.Eh;
+  for (int r = 0; r < a.R; ++r)
+    if (s.repe[j * a.R + r] == e) {
+      q = s.repq[j * a.R + r];
+      grp = a.Eh + r;
     }
+}
+
+// Flows of eq. (1) with exact quotas: every host receives exactly its quota.
+// Own rank first (a = 0), then each cost level, hosts in ascending rank taking
+// from sources in ascending rank.  Leaves this lane's column of Mw.
+__device__ void flows_exact(const PlanArgs& a, PlannerSmem& s, int e, int h0,
+                            unsigned hostmask, int nh, int d, int lane, int32_t* Mw,
+                            int32_t* qw) {
+  const int P = a.P, gpn = a.gpn;
+  int dres = d;
+  if (lane < P && ((hostmask >> lane) & 1u)) {
+    int q, grp;
+    host_quota(a, s, e, h0, lane, q, grp);
     const int my_t = __popc(hostmask & ((1u << lane) - 1u));
-    const int take = min(dres, q);  // phase 0: the host's own rank, a = 0
+    const int take = min(dres, q);  // the host's own rank, a = 0
     Mw[my_t * 32 + lane] = take;
     dres -= take;
     qw[my_t] = q - take;
@@ -355,6 +356,77 @@ __device__ long long transport_warp(const PlanArgs& a, PlannerSmem& s, int e, in
     }
   }
   if (__any_sync(kFull, dres != 0) && lane == 0) atomicExch(&s.misc[kMiscErr], 1);
+}
+
+// Flows of eq. (1) within its band: host j of quota q receives lo..hi rows,
+// lo/hi = q -/+ floor(q * cfix / 2^20).  The slack sum(q) - sum(lo) is what
+// may go above the lower bounds in total.  1: own rank up to lo; 2: hosts in
+// ascending rank take more own rows, up to hi, while slack lasts; 3: each cost
+// level, hosts in ascending rank, sources in ascending rank: up to lo, then up
+// to hi while slack lasts.  Lane j keeps host j's bounds and receipt; returns
+// the receipt (0 on other lanes) and its group in *grp_out.
+__device__ int flows_band(const PlanArgs& a, PlannerSmem& s, int e, int h0, unsigned hostmask,
+                          int nh, int d, int lane, int32_t* Mw, int* grp_out) {
+  const int P = a.P, gpn = a.gpn;
+  const bool host = lane < P && ((hostmask >> lane) & 1u);
+  const int my_t = __popc(hostmask & ((1u << lane) - 1u));
+  int dres = d, lo = 0, hi = 0, recv = 0, dl = 0, grp = -1;
+  if (host) {
+    int q;
+    host_quota(a, s, e, h0, lane, q, grp);
+    dl = int((long long)q * a.cfix >> 20);
+    lo = q - dl;
+    hi = q + dl;
+    recv = min(dres, lo);  // 1: own rank up to the lower bound
+    dres -= recv;
+  }
+  int slack = int(__reduce_add_sync(kFull, unsigned(dl)));
+  {  // 2: own rank into the band, hosts in ascending rank
+    const int want = host ? min(dres, hi - recv) : 0;
+    const int inc = warp_incl_scan(want, lane);
+    const int take = max(0, min(want, slack - (inc - want)));
+    dres -= take;
+    recv += take;
+    slack -= int(__reduce_add_sync(kFull, unsigned(take)));
+  }
+  if (host) Mw[my_t * 32 + lane] = recv;
+  __syncwarp();
+  const int nlev = gpn > 1 ? 2 : 1;
+  for (int l = 0; l < nlev; ++l) {  // 3: the other ranks, by cost level
+    const int lev = l == 0 ? 1 : 4;
+    unsigned hm = hostmask;
+    for (int t = 0; t < nh; ++t) {
+      const int j = __ffs(hm) - 1;
+      hm &= hm - 1u;
+      const int rj = __shfl_sync(kFull, recv, j);
+      const int loj = __shfl_sync(kFull, lo, j);
+      const int hij = __shfl_sync(kFull, hi, j);
+      const int need = max(loj - rj, 0);
+      const int avail = need + min(hij - max(rj, loj), slack);
+      const int v = (lane < P && cost_a(lane, j, gpn) == lev) ? dres : 0;
+      const int inc = warp_incl_scan(v, lane);
+      const int take = max(0, min(v, avail - (inc - v)));
+      const int tot = int(__reduce_add_sync(kFull, unsigned(take)));
+      Mw[t * 32 + lane] += take;
+      dres -= take;
+      if (lane == j) recv += tot;
+      slack -= max(tot - need, 0);
+    }
+  }
+  __syncwarp();
+  const bool bad = dres != 0 || (host && (recv < lo || recv > hi));
+  if (__any_sync(kFull, bad) && lane == 0) atomicExch(&s.misc[kMiscErr], 1);
+  *grp_out = grp;
+  return host ? recv : 0;
+}
+
+// From the flows in Mw: the locality cost of this source lane, and its
+// segments of expert e in host order (a ascending, then rank), each (end
+// position among the source's entries of e, first destination row).
+__device__ long long emit_segments(const PlanArgs& a, const PlannerSmem& s, int e, int h0,
+                                   unsigned hostmask, int nh, int lane, int32_t* Mw,
+                                   int2* seg) {
+  const int P = a.P, R = a.R, Eh = a.Eh, G = Eh + R, gpn = a.gpn;
   long long cost = 0;
   {
     unsigned hm = hostmask;
@@ -397,9 +469,52 @@ __device__ long long transport_warp(const PlanArgs& a, PlannerSmem& s, int e, in
   return cost;
 }
 
-// One instance per greedy mode (kMode: 0 room, 1 local, 2 kept placement), so
-// each instance carries only the greedy loop it runs.
-template <int kMode>
+// Transport of eq. (1) for expert e, run by one warp, lane = source rank.
+// kEmit: write the source lane's segments of e into the segment table and
+// return the lane's share of the locality cost.  Otherwise (banded plans
+// only) record each host's receipt in s.cu[j][grp + 1]; the group offsets
+// are known only once every expert's receipts are.
+template <bool kBand, bool kEmit>
+__device__ long long transport_warp(const PlanArgs& a, PlannerSmem& s, int e, int lane,
+                                    int32_t* Mw, int32_t* qw) {
+  const int P = a.P, Eh = a.Eh, G = Eh + a.R, gpn = a.gpn;
+  const int h0 = e / Eh;
+  const unsigned hold = s.hold[e];
+  const int d = lane < P ? s.cnt[lane * a.E + e] : 0;
+  int2* seg = a.seg + int64_t(lane) * a.seg_width + s.hoff[e];
+  if (hold == 0u) {
+    // the home rank is the only host: every source sends it all its rows
+    if (!kEmit) {
+      if (lane == 0) s.cu[h0 * (G + 1) + (e - h0 * Eh) + 1] = s.hq[e];
+      return 0;
+    }
+    const int inc = warp_incl_scan(d, lane);
+    if (lane < P)
+      seg[0] = make_int2(d, h0 * a.cap + s.cu[h0 * (G + 1) + (e - h0 * Eh)] + inc - d);
+    return (long long)cost_a(lane, h0, gpn) * d;
+  }
+  const unsigned hostmask = hold | (1u << h0);
+  const int nh = __popc(hostmask);
+  for (int t = 0; t < nh; ++t) Mw[t * 32 + lane] = 0;
+  __syncwarp();
+  if (kBand) {
+    int grp;
+    const int recv = flows_band(a, s, e, h0, hostmask, nh, d, lane, Mw, &grp);
+    if (!kEmit) {
+      if (lane < P && ((hostmask >> lane) & 1u)) s.cu[lane * (G + 1) + grp + 1] = recv;
+      __syncwarp();
+      return 0;
+    }
+  } else {
+    flows_exact(a, s, e, h0, hostmask, nh, d, lane, Mw, qw);
+  }
+  return emit_segments(a, s, e, h0, hostmask, nh, lane, Mw, seg);
+}
+
+// One instance per greedy mode (kMode: 0 room, 1 local, 2 kept placement) and
+// transport (kBand: quotas exact, or within eq. (1)'s band), so that each
+// instance carries only the code it runs.
+template <int kMode, bool kBand>
 __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
   extern __shared__ __align__(16) char smem_raw[];
   __shared__ unsigned long long s_cost;
@@ -516,32 +631,53 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
       }
     }
   }
-  // cu_seqlens: exclusive prefix of each rank's group receipts (exact quotas)
+  int32_t* Mw = s.M + warp * 32 * 32;
+  int32_t* qw = s.q + warp * 32;
+  // cu_seqlens: exclusive prefix of each rank's group receipts.  Exact quotas
+  // are the receipts; in a band they are known after a first transport pass.
+  if (kBand)
+    for (int x = tid; x < P * (G + 1); x += kPlanThreads) s.cu[x] = 0;
+  __syncthreads();
+  if (kBand)
+    for (int k = warp; k < E; k += kPlanWarps)
+      transport_warp<true, false>(a, s, s.order[k], lane, Mw, qw);
+  __syncthreads();
   for (int j = warp; j < P; j += kPlanWarps) {
     int carry = 0;
     int32_t* cu = s.cu + j * (G + 1);
-    if (lane == 0) cu[0] = 0;
     for (int g0 = 0; g0 < G; g0 += 32) {
       const int g = g0 + lane;
       int v = 0;
-      if (g < G) v = g < Eh ? s.hq[j * Eh + g] : s.repq[j * R + (g - Eh)];
+      if (g < G) {
+        if (kBand)
+          v = cu[g + 1];
+        else
+          v = g < Eh ? s.hq[j * Eh + g] : s.repq[j * R + (g - Eh)];
+      }
       const int inc = warp_incl_scan(v, lane);
+      __syncwarp();
       if (g < G) cu[g + 1] = carry + inc;
       carry += __shfl_sync(kFull, inc, 31);
     }
+    if (lane == 0) cu[0] = 0;
   }
   __syncthreads();
+  if (kBand && warp == 0) {
+    const int v = lane < P ? s.cu[lane * (G + 1) + G] : 0;
+    if (lane < P) a.load_after[lane] = v;
+    const int mx = int(__reduce_max_sync(kFull, unsigned(v)));
+    if (lane == 0) s.misc[kMiscRecv] = mx;
+  }
   for (int x = tid; x < P * (G + 1); x += kPlanThreads) a.cu_seqlens[x] = s.cu[x];
   for (int e = tid; e <= E; e += kPlanThreads) a.hoff[e] = s.hoff[e];
+  __syncthreads();
 
-  const bool capacity = max_load > a.cap;
+  const int rows_max = kBand ? s.misc[kMiscRecv] : max_load;
+  const bool capacity = rows_max > a.cap;
   long long cost_part = 0;
-  if (!capacity) {
-    int32_t* Mw = s.M + warp * 32 * 32;
-    int32_t* qw = s.q + warp * 32;
+  if (!capacity)
     for (int k = warp; k < E; k += kPlanWarps)
-      cost_part += transport_warp(a, s, s.order[k], lane, Mw, qw);
-  }
+      cost_part += transport_warp<kBand, true>(a, s, s.order[k], lane, Mw, qw);
   cost_part = warp_sum64(cost_part);
   if (lane == 0) atomicAdd(&s_cost, (unsigned long long)cost_part);
   __syncthreads();
@@ -554,7 +690,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
     else if (max_load > T)
       status = ZB_WARN_UNBALANCED;
     a.stats[ZB_STAT_STATUS] = status;
-    a.stats[ZB_STAT_MAX_LOAD] = max_load;
+    a.stats[ZB_STAT_MAX_LOAD] = rows_max;
     a.stats[ZB_STAT_N_REPLICAS] = s.misc[kMiscNrep];
     a.stats[ZB_STAT_N_ITERS] = s.misc[kMiscIters];
     a.stats[ZB_STAT_WATER_LEVEL] = T;
@@ -662,7 +798,7 @@ cudaError_t launch_hist(const PlanArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-template <int kMode>
+template <int kMode, bool kBand>
 cudaError_t launch_planner_mode(const PlanArgs& a, size_t smem, cudaStream_t s) {
   static bool configured[64] = {};
   int dev = 0;
@@ -670,19 +806,24 @@ cudaError_t launch_planner_mode(const PlanArgs& a, size_t smem, cudaStream_t s) 
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    err = cudaFuncSetAttribute(k_planner<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               200 * 1024);
+    err = cudaFuncSetAttribute(k_planner<kMode, kBand>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     if (err != cudaSuccess) return err;
     configured[dev] = true;
   }
-  k_planner<kMode><<<1, kPlanThreads, smem, s>>>(a);
+  k_planner<kMode, kBand><<<1, kPlanThreads, smem, s>>>(a);
   return cudaGetLastError();
 }
 
+template <bool kBand>
+cudaError_t launch_planner_band(const PlanArgs& a, size_t smem, cudaStream_t s) {
+  if (a.placement) return launch_planner_mode<2, kBand>(a, smem, s);
+  if (a.policy == ZB_POLICY_LOCAL) return launch_planner_mode<ZB_POLICY_LOCAL, kBand>(a, smem, s);
+  return launch_planner_mode<ZB_POLICY_ROOM, kBand>(a, smem, s);
+}
+
 cudaError_t launch_planner(const PlanArgs& a, size_t smem, cudaStream_t s) {
-  if (a.placement) return launch_planner_mode<2>(a, smem, s);
-  if (a.policy == ZB_POLICY_LOCAL) return launch_planner_mode<ZB_POLICY_LOCAL>(a, smem, s);
-  return launch_planner_mode<ZB_POLICY_ROOM>(a, smem, s);
+  return a.relax ? launch_planner_band<true>(a, smem, s) : launch_planner_band<false>(a, smem, s);
 }
 
 cudaError_t launch_assign(const PlanArgs& a, cudaStream_t s) {

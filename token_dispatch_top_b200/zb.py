@@ -9,6 +9,7 @@ raises.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 from dataclasses import dataclass
 
@@ -47,7 +48,8 @@ class _Cfg(ctypes.Structure):
     _fields_ = [("P", ctypes.c_int), ("E", ctypes.c_int), ("K", ctypes.c_int),
                 ("S", ctypes.c_int), ("H", ctypes.c_int), ("R", ctypes.c_int),
                 ("C", ctypes.c_float), ("gpus_per_node", ctypes.c_int),
-                ("cap_rows", ctypes.c_int), ("policy", ctypes.c_int)]
+                ("cap_rows", ctypes.c_int), ("policy", ctypes.c_int),
+                ("relax", ctypes.c_int)]
 
 
 class _Plan(ctypes.Structure):
@@ -106,12 +108,19 @@ class Config:
     R: int
     C: float = 0.0
     gpus_per_node: int = 1
-    cap_rows: int | None = None  # default S*K
+    cap_rows: int | None = None  # default S*K, or floor((1+C) S*K) with relax
     policy: int = 0              # POLICY_ROOM or POLICY_LOCAL
+    relax: int = 0               # 1: receipts within q +- floor(C q), eq. (1)
 
     @property
     def cap(self) -> int:
-        return self.S * self.K if self.cap_rows is None else self.cap_rows
+        if self.cap_rows is not None:
+            return self.cap_rows
+        sk = self.S * self.K
+        if not self.relax:
+            return sk
+        c20 = int(math.floor(float(ctypes.c_float(self.C).value) * 1048576.0))
+        return sk + ((sk * c20) >> 20)
 
     @property
     def Eh(self) -> int:
@@ -119,7 +128,7 @@ class Config:
 
     def c(self) -> _Cfg:
         return _Cfg(self.P, self.E, self.K, self.S, self.H, self.R, float(self.C),
-                    self.gpus_per_node, self.cap, self.policy)
+                    self.gpus_per_node, self.cap, self.policy, self.relax)
 
 
 def validate(cfg: Config) -> int:
