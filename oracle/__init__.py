@@ -46,7 +46,7 @@ class _Cfg(ctypes.Structure):
                 ("S", ctypes.c_int), ("H", ctypes.c_int), ("R", ctypes.c_int),
                 ("C", ctypes.c_double), ("gpus_per_node", ctypes.c_int),
                 ("cap_rows", ctypes.c_int), ("policy", ctypes.c_int),
-                ("relax", ctypes.c_int)]
+                ("relax", ctypes.c_int), ("repair", ctypes.c_int)]
 
 
 _P32 = ctypes.POINTER(ctypes.c_int32)
@@ -58,7 +58,7 @@ class _Out(ctypes.Structure):
                 ("cu_seqlens", _P32), ("dst_row", _P32), ("row_src", _P32), ("M", _P32),
                 ("locality_cost", ctypes.c_int64), ("max_load", ctypes.c_int32),
                 ("n_replicas", ctypes.c_int32), ("n_iters", ctypes.c_int32),
-                ("water_level", ctypes.c_int32)]
+                ("water_level", ctypes.c_int32), ("repaired", ctypes.c_int32)]
 
 
 _lib = None
@@ -107,6 +107,7 @@ class Config:
     cap_rows: int | None = None
     policy: int = 0  # receiver choice: 0 most room, 1 most local rows
     relax: int = 0   # 1: hosts receive within q +- floor(C q) (eq. (1))
+    repair: int = 0  # 1: quota repair between rank pairs (HALO-Q stage 4)
 
     def cap(self) -> int:
         if self.cap_rows is not None:
@@ -119,7 +120,7 @@ class Config:
 
     def c(self) -> _Cfg:
         return _Cfg(self.P, self.E, self.K, self.S, self.H, self.R, float(self.C),
-                    self.gpus_per_node, self.cap(), self.policy, self.relax)
+                    self.gpus_per_node, self.cap(), self.policy, self.relax, self.repair)
 
 
 def _ptr(a: np.ndarray):
@@ -157,14 +158,15 @@ def plan(cfg: Config, ids: np.ndarray, want_M: bool = True,
     out = _Out(*[_ptr(r[k]) for k in ("cnt", "rep_expert", "rep_quota", "home_quota",
                                        "load_before", "load_after", "cu_seqlens",
                                        "dst_row", "row_src")],
-               _ptr(r["M"]) if want_M else _P32(), 0, 0, 0, 0, 0)
+               _ptr(r["M"]) if want_M else _P32(), 0, 0, 0, 0, 0, 0)
     if placement is None:
         st = lib.zbo_plan(ctypes.byref(cfg.c()), _ptr(ids), ctypes.byref(out))
     else:
         pl = np.ascontiguousarray(placement, dtype=np.int32).reshape(P, R)
         st = lib.zbo_plan_placed(ctypes.byref(cfg.c()), _ptr(ids), _ptr(pl), ctypes.byref(out))
     r.update(status=int(st), locality_cost=int(out.locality_cost), max_load=int(out.max_load),
-             n_replicas=int(out.n_replicas), n_iters=int(out.n_iters), T=int(out.water_level))
+             n_replicas=int(out.n_replicas), n_iters=int(out.n_iters), T=int(out.water_level),
+             repaired=int(out.repaired))
     return r
 
 

@@ -40,6 +40,7 @@
  *    relax = 1 each host of quota q receives between q - dl and q + dl rows,
  *    dl = floor(q * C) with C taken to 20 fractional bits, and the receive
  *    buffers hold floor((1+C) T) rows [ZEPP 4.1, eq. (1)]; see transport().
+ *  - quota repair (repair = 1) [ISER, HALO-Q stage 4]: see repair_quotas().
  *  - rows inside a group are ordered by (source rank, flat index s*K+k).
  *  - combine: acc = +0.0f; acc = fmaf(w_k, y_k, acc) for k = 0..K-1; the
  *    result is rounded to bf16 to nearest, ties to even.
@@ -71,6 +72,7 @@ typedef struct {
   int cap_rows;      /* rows of each rank's receive buffer (>= S*K) */
   int policy;        /* receiver choice: 0 most room, 1 most local rows */
   int relax;         /* 0 quotas met exactly; 1 within the band of eq. (1) */
+  int repair;        /* 1: quota repair between rank pairs after the greedy */
 } zbo_config;
 
 typedef struct {
@@ -89,6 +91,7 @@ typedef struct {
   int32_t n_replicas;
   int32_t n_iters;
   int32_t water_level;
+  int32_t repaired;     /* rows moved by quota repair, per direction */
 } zbo_plan_out;
 
 /* ---------------------------------------------------------------- helpers */
@@ -120,6 +123,7 @@ int zbo_validate(const zbo_config *c) {
   if ((int64_t)c->P * c->cap_rows > INT32_MAX) return ZBO_ERR_INVALID;
   if (c->policy != 0 && c->policy != 1) return ZBO_ERR_INVALID;
   if (c->relax != 0 && c->relax != 1) return ZBO_ERR_INVALID;
+  if (c->repair != 0 && c->repair != 1) return ZBO_ERR_INVALID;
   return ZBO_OK;
 }
 
@@ -321,6 +325,73 @@ int zbo_placement_valid(const zbo_config *c, const int32_t *rep_expert) {
   return 1;
 }
 
+/* ------------------------------------------------ quota repair (stage 4) */
+
+/* q_r^e: the quota of rank r for expert e (0 when r holds no copy), and a
+ * pointer to where it is kept. */
+static int32_t *quota_ref(const zbo_config *c, int r, int e, int32_t *home_quota,
+                          const int32_t *rep_expert, int32_t *rep_quota) {
+  if (home_of(c, e) == r) return &home_quota[e];
+  for (int s = 0; s < c->R; s++)
+    if (rep_expert[r * c->R + s] == e) return &rep_quota[r * c->R + s];
+  return NULL;
+}
+
+/* Quota repair [ISER, HALO-Q stage 4: a circle-method tournament over
+ * disjoint rank pairs that cancels opposite token flows].  For ranks i and j
+ * that both hold expert e, rank i has a surplus of e (its own rows beyond its
+ * quota, which must leave it) and j a spare (quota beyond its own rows, which
+ * other ranks must fill).  When i has surplus of e where j has spare, and j
+ * has surplus of e' where i has spare, moving m rows of quota of e from j to i
+ * and m of e' from i to j cancels m rows each way and leaves both loads as
+ * they are.  Per pair, the cancellable amounts a_e = min(surplus_i^e,
+ * spare_j^e) and b_e' = min(surplus_j^e', spare_i^e') are consumed in
+ * ascending expert order up to min(sum a, sum b).  The pairs come from the
+ * circle method: ranks 0..P'-1 (P' = P rounded up to even; rank P is a bye),
+ * round r = 0..P'-2 pairs P'-1 with r and (r+k) mod (P'-1) with (r-k) mod
+ * (P'-1) for k = 1..P'/2-1; each pair is handled with i the lower rank.
+ * Pairs within a round are disjoint.  Returns the rows moved per direction. */
+static int32_t repair_quotas(const zbo_config *c, const int32_t *cnt, int32_t *home_quota,
+                             const int32_t *rep_expert, int32_t *rep_quota) {
+  const int P = c->P, E = c->E, Pp = P + (P & 1);
+  int32_t moved = 0;
+  int32_t *a = malloc(sizeof(int32_t) * (size_t)E), *b = malloc(sizeof(int32_t) * (size_t)E);
+  for (int r = 0; r < Pp - 1; r++)
+    for (int k = 0; k < Pp / 2; k++) {
+      int x = k == 0 ? Pp - 1 : (r + k) % (Pp - 1);
+      int y = k == 0 ? r : (r - k + (Pp - 1)) % (Pp - 1);
+      if (x >= P || y >= P) continue; /* the bye */
+      int i = x < y ? x : y, j = x < y ? y : x;
+      int64_t sa = 0, sb = 0;
+      for (int e = 0; e < E; e++) {
+        a[e] = b[e] = 0;
+        int32_t *qi = quota_ref(c, i, e, home_quota, rep_expert, rep_quota);
+        int32_t *qj = quota_ref(c, j, e, home_quota, rep_expert, rep_quota);
+        if (!qi || !qj) continue;
+        int32_t di = cnt[(size_t)i * E + e], dj = cnt[(size_t)j * E + e];
+        int32_t sur_i = di > *qi ? di - *qi : 0, spare_i = *qi > di ? *qi - di : 0;
+        int32_t sur_j = dj > *qj ? dj - *qj : 0, spare_j = *qj > dj ? *qj - dj : 0;
+        a[e] = sur_i < spare_j ? sur_i : spare_j;
+        b[e] = sur_j < spare_i ? sur_j : spare_i;
+        sa += a[e];
+        sb += b[e];
+      }
+      int64_t m = sa < sb ? sa : sb, ra = m, rb = m;
+      for (int e = 0; e < E && (ra > 0 || rb > 0); e++) {
+        int32_t *qi = quota_ref(c, i, e, home_quota, rep_expert, rep_quota);
+        int32_t *qj = quota_ref(c, j, e, home_quota, rep_expert, rep_quota);
+        int32_t ta = (int32_t)(a[e] < ra ? a[e] : ra); /* e: quota from j to i */
+        int32_t tb = (int32_t)(b[e] < rb ? b[e] : rb); /* e: quota from i to j */
+        if (ta) { *qi += ta; *qj -= ta; ra -= ta; }
+        if (tb) { *qj += tb; *qi -= tb; rb -= tb; }
+      }
+      moved += (int32_t)m;
+    }
+  free(a);
+  free(b);
+  return moved;
+}
+
 /* ------------------------- step 3: transport, groups, cu_seqlens, rows */
 
 typedef struct { int rank, group; int32_t quota; } host_t;
@@ -464,6 +535,10 @@ int zbo_plan_placed(const zbo_config *c, const int32_t *ids, const int32_t *plac
     greedy_place(c, out->cnt, T, out->load_after, out->home_quota, out->rep_expert,
                  out->rep_quota, &out->n_iters);
   }
+
+  out->repaired = 0;
+  if (c->repair)
+    out->repaired = repair_quotas(c, out->cnt, out->home_quota, out->rep_expert, out->rep_quota);
 
   out->max_load = 0;
   out->n_replicas = 0;

@@ -22,7 +22,7 @@ def _cfg(d):
     return oracle.Config(P=d["P"], E=d["E"], K=d["K"], S=d["S"], H=d["H"], R=d["R"],
                          C=d.get("C", 0.0), gpus_per_node=d.get("gpus_per_node", 1),
                          cap_rows=d.get("cap_rows"), policy=d.get("policy", 0),
-                         relax=d.get("relax", 0))
+                         relax=d.get("relax", 0), repair=d.get("repair", 0))
 
 
 def _examples():
@@ -33,7 +33,8 @@ def _examples():
 def test_hand_examples(ex):
     cfg = _cfg(ex["cfg"])
     ids = np.array(ex["ids"], np.int32).reshape(cfg.P, cfg.S, cfg.K)
-    p = oracle.plan(cfg, ids)
+    pl = np.array(ex["placement"], np.int32) if "placement" in ex else None
+    p = oracle.plan(cfg, ids, placement=pl)
     exp = ex["expect"]
     assert p["status"] == exp["status"]
     assert p["T"] == exp["T"]
@@ -52,8 +53,11 @@ def test_hand_examples(ex):
     if "cap" in exp:
         assert cfg.cap() == exp["cap"]
     if "locality_cost_exact_quotas" in exp:
-        cfg0 = _cfg(dict(ex["cfg"], relax=0))
-        assert oracle.plan(cfg0, ids)["locality_cost"] == exp["locality_cost_exact_quotas"]
+        cfg0 = _cfg(dict(ex["cfg"], relax=0, repair=0))
+        assert oracle.plan(cfg0, ids, placement=pl)["locality_cost"] == \
+            exp["locality_cost_exact_quotas"]
+    if "repaired" in exp:
+        assert p["repaired"] == exp["repaired"]
     if "status_with_cap_rows_3" in exp:
         cfg.cap_rows = 3
         assert oracle.plan(cfg, ids)["status"] == exp["status_with_cap_rows_3"]
