@@ -381,6 +381,37 @@ def run_ours(args, wl, rank, world, local_rank):
         "locality_cost_exact": int(st_x[zb.STAT_LOCALITY_COST])}
     del plan_b
 
+    # ---- quota repair (HALO-Q stage 4) on a kept placement that puts the
+    # R = 4 hottest foreign experts on every rank, timed apart from the step
+    R4 = min(4, wl.P - 1)
+    Te = np.bincount(ids_np.ravel(), minlength=wl.E)
+    pl_np = np.full((wl.P, R4), -1, np.int32)
+    for j in range(wl.P):
+        hot = [e for e in np.argsort(-Te, kind="stable") if e // (wl.E // wl.P) != j][:R4]
+        pl_np[j, :len(hot)] = hot
+    pl_d = torch.from_numpy(pl_np).to(dev)
+    rep = {"what": f"zb_plan_placed with every rank holding the {R4} hottest foreign experts, "
+                   "without and with quota repair (ISER-MoE HALO-Q stage 4); not part of the step"}
+    for tag, flag in (("kept", 0), ("repaired", 1)):
+        cfg_r = dataclasses.replace(cfg, R=R4, repair=flag, cap_rows=2 * wl.S * wl.K)
+        plan_r = zb.Plan(cfg_r, dev, with_row_src=False)
+        zb.plan_placed(plan_r, ids, pl_d)
+        torch.cuda.synchronize()
+        r_ms = []
+        for _ in range(max(20, min(args.steps, 100))):
+            flush_l2()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            zb.plan_placed(plan_r, ids, pl_d)
+            a1.record(stream)
+            a1.synchronize()
+            r_ms.append(a0.elapsed_time(a1))
+        st_r = plan_r.stats.cpu().numpy()
+        rep[tag] = {"status": int(st_r[zb.STAT_STATUS]), "plan_ms": statistics.median(r_ms),
+                    "locality_cost": int(st_r[zb.STAT_LOCALITY_COST]),
+                    "rows_repaired": int(st_r[zb.STAT_REPAIRED])}
+        del plan_r
+
     # ---- end to end through the public API, pinned host buffers.  Every step
     # copies its ids, gates and hidden rows host->device, runs plan, dispatch
     # and combine, and copies its combined rows and plan status back.  Copies
@@ -504,7 +535,7 @@ def run_ours(args, wl, rank, world, local_rank):
             "dispatch_ms": statistics.median(d_ms),
             "dispatch_gbs": (wl.tokens * wl.H * 2 + rows_merged * wl.H * 2 + wl.N * 4)
             / statistics.median(d_ms) / 1e6},
-            "banded_plan": banded},
+            "banded_plan": banded, "quota_repair": rep},
         "wall_s": wall,
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,

@@ -85,7 +85,18 @@ extern "C" {
  *         total slack (sum of dl) lasts, then the other ranks by cost level.
  *         When the quota loads reach T, a rank receives at most
  *         T + floor(T * floor(C * 2^20) / 2^20) = floor((1+C) T) rows; size
- *         cap_rows for that (a plan needing more is ZB_ERR_CAPACITY). */
+ *         cap_rows for that (a plan needing more is ZB_ERR_CAPACITY).
+ *   repair  1: after the greedy (or the kept placement's quotas), quota
+ *         repair between rank pairs (ISER-MoE, HALO-Q stage 4).  Ranks i and
+ *         j that both hold experts e and e' cancel opposite flows: where i's
+ *         own rows of e exceed its quota (surplus) and j's quota of e exceeds
+ *         j's own rows (spare), and the reverse holds for e', m rows of quota
+ *         of e move from j to i and m of e' from i to j.  Both loads are
+ *         unchanged; 2m more rows are served on their own rank.  Per pair,
+ *         m = min(sum_e min(surplus_i, spare_j), sum_e min(surplus_j, spare_i)),
+ *         consumed in ascending expert order.  Pairs come from the circle
+ *         method over P rounded up to even (a bye for odd P), one round after
+ *         another.  Filled slots may end with quota 0.  0: no repair. */
 #define ZB_POLICY_ROOM 0
 #define ZB_POLICY_LOCAL 1
 typedef struct zb_config {
@@ -95,6 +106,7 @@ typedef struct zb_config {
   int cap_rows;
   int policy;
   int relax;
+  int repair;
 } zb_config;
 
 /* Indices into plan->stats (int64). */
@@ -105,13 +117,15 @@ typedef struct zb_config {
 #define ZB_STAT_WATER_LEVEL 4   /* T = ceil(sum_r L_r / P) */
 #define ZB_STAT_LOCALITY_COST 5 /* sum_{e,i,j} a_ij M^e_ij */
 #define ZB_STAT_BAD_IDS 6       /* count of ids outside [0, E) */
+#define ZB_STAT_REPAIRED 7      /* rows moved by quota repair, per direction */
 #define ZB_STATS_LEN 8
 
 /* The plan: caller-allocated device buffers that zb_plan fills and
  * zb_dispatch / zb_combine read.  Shapes (int32 unless stated):
  *   cnt         [P][E]        cnt[i][e] = #{(s,k): ids[i,s,k] = e}
  *   rep_expert  [P][R]        expert held by helper slot (j, r), -1 = empty
- *   rep_quota   [P][R]        rows that slot receives (0 if empty)
+ *   rep_quota   [P][R]        rows that slot receives (0 if empty; with
+ *                             repair, a filled slot may also have 0)
  *   home_quota  [E]           rows the home copy of e receives
  *   load_before [P]           L_j = rows homed on j before planning
  *   load_after  [P]           rows rank j receives after planning (its

@@ -13,9 +13,10 @@ PLAN_KEYS = ("cnt", "rep_expert", "rep_quota", "home_quota", "load_before", "loa
 SENTINEL = 0x7E11  # bf16 bit pattern marking rows nobody may write
 
 
-def cfgs(wl: synth.Workload, cap_rows=None, policy=0, relax=0, C=None):
+def cfgs(wl: synth.Workload, cap_rows=None, policy=0, relax=0, C=None, repair=0):
     kw = dict(P=wl.P, E=wl.E, K=wl.K, S=wl.S, H=wl.H, R=wl.R, C=wl.C if C is None else C,
-              gpus_per_node=wl.gpus_per_node, cap_rows=cap_rows, policy=policy, relax=relax)
+              gpus_per_node=wl.gpus_per_node, cap_rows=cap_rows, policy=policy, relax=relax,
+              repair=repair)
     return zb.Config(**kw), oracle.Config(**kw)
 
 
@@ -54,6 +55,7 @@ def assert_plan_equal(g: dict, o: dict, status: int, rows=True):
     assert st[zb.STAT_WATER_LEVEL] == o["T"]
     assert st[zb.STAT_N_REPLICAS] == o["n_replicas"]
     assert st[zb.STAT_N_ITERS] == o["n_iters"]
+    assert st[zb.STAT_REPAIRED] == o["repaired"]
     for k in PLAN_KEYS:
         np.testing.assert_array_equal(g[k], o[k], err_msg=k)
     if status >= 0:

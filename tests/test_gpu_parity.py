@@ -78,9 +78,16 @@ def test_hand_examples(dev, ex):
     d = ex["cfg"]
     kw = dict(P=d["P"], E=d["E"], K=d["K"], S=d["S"], H=d["H"], R=d["R"], C=d.get("C", 0.0),
               gpus_per_node=d.get("gpus_per_node", 1), cap_rows=d.get("cap_rows"),
-              policy=d.get("policy", 0), relax=d.get("relax", 0))
+              policy=d.get("policy", 0), relax=d.get("relax", 0), repair=d.get("repair", 0))
     zc, oc = zb.Config(**kw), oracle.Config(**kw)
     ids = np.array(ex["ids"], np.int32).reshape(zc.P, zc.S, zc.K)
+    if "placement" in ex:  # a kept placement: the plan tables through zb_plan_placed
+        pl = np.array(ex["placement"], np.int32)
+        p = zb.Plan(zc, dev)
+        zb.plan_placed(p, torch.from_numpy(ids).to(dev), torch.from_numpy(pl).to(dev))
+        status, _ = zb.plan_status(p)
+        assert_plan_equal(plan_tables(p), oracle.plan(oc, ids, placement=pl), status)
+        return
     rng = np.random.default_rng(0)
     w = rng.dirichlet(np.ones(zc.K), size=(zc.P, zc.S)).astype(np.float32)
     full_parity(zc, oc, ids, w, _rand_bits(rng, (zc.P, zc.S, zc.H)),

@@ -108,6 +108,8 @@ struct PlannerSmem {
   int32_t* q;      // [warps][32 hosts] remaining quota in transport
   int32_t* misc;   // [16]
   int32_t* M;      // [warps][32 hosts][32 sources]
+  int16_t* qidx;   // [P*E] quota repair only: where rank r keeps its quota of
+                   // e (e: hq[e]; E + x: repq[x]; -1: no copy)
 };
 
 __device__ PlannerSmem carve(char* base, const PlanArgs& a) {
@@ -123,13 +125,15 @@ __device__ PlannerSmem carve(char* base, const PlanArgs& a) {
   s.order = p; p += a.E;
   s.q = p; p += kPlanWarps * 32;
   s.misc = p; p += 16;
-  s.M = p;
+  s.M = p; p += kPlanWarps * 32 * 32;
+  s.qidx = reinterpret_cast<int16_t*>(p);
   return s;
 }
 
 enum {
   kMiscT = 0, kMiscMax = 1, kMiscNrep = 2, kMiscIters = 3, kMiscBad = 4, kMiscErr = 5,
-  kMiscRecv = 6  // banded plans: the most rows any rank receives
+  kMiscRecv = 6,     // banded plans: the most rows any rank receives
+  kMiscRepaired = 7  // rows moved by quota repair, per direction
 };
 
 // Greedy replica placement, run by one warp; lane r holds rank r's load,
@@ -299,6 +303,76 @@ __device__ void greedy_placed_warp(const PlanArgs& a, PlannerSmem& s, int T, int
     s.misc[kMiscNrep] = nrep;
     s.misc[kMiscIters] = iters;
   }
+}
+
+// Quota of the copy at quota index x (x < E: home quota of x; else helper
+// slot x - E).
+__device__ __forceinline__ int32_t& quota_at(const PlanArgs& a, PlannerSmem& s, int x) {
+  return x < a.E ? s.hq[x] : s.repq[x - a.E];
+}
+
+// Quota repair of one rank pair (i < j), run by one warp (ISER-MoE, HALO-Q
+// stage 4).  The experts both ranks hold are i's helper copies of experts j
+// holds, plus j's helper copies of experts homed on i: lane c < R takes i's
+// slot c, lane R + c takes j's slot c (two rounds of lanes when 2R > 32).
+// For each, a = min(surplus_i, spare_j) and b = min(surplus_j, spare_i);
+// m = min(sum a, sum b) rows of quota move each way.  The side whose sum
+// exceeds m is consumed in ascending expert order, the other in full.
+// Both loads are unchanged.
+__device__ void repair_pair_warp(const PlanArgs& a, PlannerSmem& s, int i, int j, int lane) {
+  const int R = a.R, E = a.E, Eh = a.Eh, nc = 2 * R;
+  const int nu = nc > 32 ? 2 : 1;
+  int ce[2], ca[2], cb[2], xi[2], xj[2];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    ce[u] = -1;
+    ca[u] = cb[u] = 0;
+    xi[u] = xj[u] = 0;
+    const int c = lane + 32 * u;
+    if (u >= nu || c >= nc) continue;
+    int e = c < R ? s.repe[i * R + c] : s.repe[j * R + (c - R)];
+    if (e < 0) continue;
+    if (c < R ? s.qidx[j * E + e] < 0 : e / Eh != i) continue;
+    ce[u] = e;
+    xi[u] = s.qidx[i * E + e];
+    xj[u] = s.qidx[j * E + e];
+    const int qi = quota_at(a, s, xi[u]), qj = quota_at(a, s, xj[u]);
+    const int di = s.cnt[i * E + e], dj = s.cnt[j * E + e];
+    ca[u] = min(max(di - qi, 0), max(qj - dj, 0));
+    cb[u] = min(max(dj - qj, 0), max(qi - di, 0));
+  }
+  const int sa = int(__reduce_add_sync(kFull, unsigned(ca[0] + ca[1])));
+  const int sb = int(__reduce_add_sync(kFull, unsigned(cb[0] + cb[1])));
+  const int m = min(sa, sb);
+  if (m == 0) return;
+  int ta[2] = {ca[0], ca[1]}, tb[2] = {cb[0], cb[1]};
+  if (sa != sb) {  // cut the larger side at m, in ascending expert order
+    const bool cut_a = sa > m;
+    int v[2] = {cut_a ? ca[0] : cb[0], cut_a ? ca[1] : cb[1]};
+    int before[2] = {0, 0};
+    for (int t = 0; t < nc; ++t) {
+      const int et = __shfl_sync(kFull, t < 32 ? ce[0] : ce[1], t & 31);
+      const int vt = __shfl_sync(kFull, t < 32 ? v[0] : v[1], t & 31);
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+        if (et >= 0 && et < ce[u]) before[u] += vt;
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int take = max(0, min(v[u], m - before[u]));
+      if (cut_a)
+        ta[u] = take;
+      else
+        tb[u] = take;
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 2; ++u)
+    if (ce[u] >= 0 && (ta[u] | tb[u])) {
+      quota_at(a, s, xi[u]) += ta[u] - tb[u];
+      quota_at(a, s, xj[u]) += tb[u] - ta[u];
+    }
+  if (lane == 0) atomicAdd(&s.misc[kMiscRepaired], m);
 }
 
 // Host j's quota for expert e and the group that receives it on j.
@@ -511,10 +585,10 @@ __device__ long long transport_warp(const PlanArgs& a, PlannerSmem& s, int e, in
   return emit_segments(a, s, e, h0, hostmask, nh, lane, Mw, seg);
 }
 
-// One instance per greedy mode (kMode: 0 room, 1 local, 2 kept placement) and
-// transport (kBand: quotas exact, or within eq. (1)'s band), so that each
-// instance carries only the code it runs.
-template <int kMode, bool kBand>
+// One instance per greedy mode (kMode: 0 room, 1 local, 2 kept placement),
+// quota repair (kRepair) and transport (kBand: quotas exact, or within eq.
+// (1)'s band), so that each instance carries only the code it runs.
+template <int kMode, bool kRepair, bool kBand>
 __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
   extern __shared__ __align__(16) char smem_raw[];
   __shared__ unsigned long long s_cost;
@@ -526,6 +600,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
   if (tid == 0) {
     s.misc[kMiscBad] = 0;
     s.misc[kMiscErr] = 0;
+    s.misc[kMiscRepaired] = 0;
     s_cost = 0ull;
   }
   __syncthreads();
@@ -599,6 +674,27 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
       greedy_warp<kMode>(a, s, T, L, lane);
   }
   __syncthreads();
+
+  if (kRepair) {
+    for (int x = tid; x < P * E; x += kPlanThreads) s.qidx[x] = -1;
+    __syncthreads();
+    for (int e = tid; e < E; e += kPlanThreads) s.qidx[(e / Eh) * E + e] = int16_t(e);
+    for (int x = tid; x < P * R; x += kPlanThreads)
+      if (s.repe[x] >= 0) s.qidx[(x / R) * E + s.repe[x]] = int16_t(E + x);
+    __syncthreads();
+    // circle method: ranks 0..Pp-1 (rank P is a bye when P is odd); round r
+    // pairs Pp-1 with r and (r+k) mod (Pp-1) with (r-k) mod (Pp-1); the pairs
+    // of a round are disjoint, one warp each
+    const int Pp = P + (P & 1);
+    for (int r = 0; r < Pp - 1; ++r) {
+      for (int k = warp; k < Pp / 2; k += kPlanWarps) {
+        const int x = k == 0 ? Pp - 1 : (r + k) % (Pp - 1);
+        const int y = k == 0 ? r : (r - k + (Pp - 1)) % (Pp - 1);
+        if (x < P && y < P) repair_pair_warp(a, s, min(x, y), max(x, y), lane);
+      }
+      __syncthreads();
+    }
+  }
 
   const int T = s.misc[kMiscT];
   const int max_load = s.misc[kMiscMax];
@@ -696,7 +792,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
     a.stats[ZB_STAT_WATER_LEVEL] = T;
     a.stats[ZB_STAT_LOCALITY_COST] = capacity ? 0 : (long long)s_cost;
     a.stats[ZB_STAT_BAD_IDS] = 0;
-    a.stats[7] = 0;
+    a.stats[ZB_STAT_REPAIRED] = s.misc[kMiscRepaired];
   }
 }
 
@@ -789,7 +885,9 @@ size_t planner_smem_bytes(const zb_config& c) {
                  size_t(c.P) * (Eh + c.R + 1) + size_t(c.E + 1) + size_t(c.E) +
                  kPlanWarps * 32 + 16;
   words += size_t(kPlanWarps) * 32 * 32;
-  return words * sizeof(int32_t);
+  size_t bytes = words * sizeof(int32_t);
+  if (c.repair) bytes += sizeof(int16_t) * size_t(c.P) * c.E;  // qidx
+  return bytes;
 }
 
 cudaError_t launch_hist(const PlanArgs& a, cudaStream_t s) {
@@ -798,7 +896,7 @@ cudaError_t launch_hist(const PlanArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-template <int kMode, bool kBand>
+template <int kMode, bool kRepair, bool kBand>
 cudaError_t launch_planner_mode(const PlanArgs& a, size_t smem, cudaStream_t s) {
   static bool configured[64] = {};
   int dev = 0;
@@ -806,24 +904,29 @@ cudaError_t launch_planner_mode(const PlanArgs& a, size_t smem, cudaStream_t s) 
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    err = cudaFuncSetAttribute(k_planner<kMode, kBand>,
+    err = cudaFuncSetAttribute(k_planner<kMode, kRepair, kBand>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     if (err != cudaSuccess) return err;
     configured[dev] = true;
   }
-  k_planner<kMode, kBand><<<1, kPlanThreads, smem, s>>>(a);
+  k_planner<kMode, kRepair, kBand><<<1, kPlanThreads, smem, s>>>(a);
   return cudaGetLastError();
 }
 
-template <bool kBand>
-cudaError_t launch_planner_band(const PlanArgs& a, size_t smem, cudaStream_t s) {
-  if (a.placement) return launch_planner_mode<2, kBand>(a, smem, s);
-  if (a.policy == ZB_POLICY_LOCAL) return launch_planner_mode<ZB_POLICY_LOCAL, kBand>(a, smem, s);
-  return launch_planner_mode<ZB_POLICY_ROOM, kBand>(a, smem, s);
+template <bool kRepair, bool kBand>
+cudaError_t launch_planner_variant(const PlanArgs& a, size_t smem, cudaStream_t s) {
+  if (a.placement) return launch_planner_mode<2, kRepair, kBand>(a, smem, s);
+  if (a.policy == ZB_POLICY_LOCAL)
+    return launch_planner_mode<ZB_POLICY_LOCAL, kRepair, kBand>(a, smem, s);
+  return launch_planner_mode<ZB_POLICY_ROOM, kRepair, kBand>(a, smem, s);
 }
 
 cudaError_t launch_planner(const PlanArgs& a, size_t smem, cudaStream_t s) {
-  return a.relax ? launch_planner_band<true>(a, smem, s) : launch_planner_band<false>(a, smem, s);
+  if (a.repair)
+    return a.relax ? launch_planner_variant<true, true>(a, smem, s)
+                   : launch_planner_variant<true, false>(a, smem, s);
+  return a.relax ? launch_planner_variant<false, true>(a, smem, s)
+                 : launch_planner_variant<false, false>(a, smem, s);
 }
 
 cudaError_t launch_assign(const PlanArgs& a, cudaStream_t s) {

@@ -60,6 +60,7 @@ int zb_validate(const zb_config* c) {
   if (int64_t(c->P) * c->cap_rows > INT32_MAX) return ZB_ERR_INVALID;
   if (c->policy != ZB_POLICY_ROOM && c->policy != ZB_POLICY_LOCAL) return ZB_ERR_INVALID;
   if (c->relax != 0 && c->relax != 1) return ZB_ERR_INVALID;
+  if (c->repair != 0 && c->repair != 1) return ZB_ERR_INVALID;
   return ZB_OK;
 }
 
@@ -86,6 +87,7 @@ int plan_impl(const zb_config* c, const int32_t* ids, const int32_t* placement,
   a.P = c->P; a.E = c->E; a.K = c->K; a.S = c->S; a.R = c->R; a.Eh = c->E / c->P;
   a.gpn = c->gpus_per_node; a.cap = c->cap_rows; a.policy = c->policy;
   a.relax = c->relax;
+  a.repair = c->repair;
   a.cfix = c->relax ? int(std::floor(double(c->C) * 1048576.0)) : 0;
   a.nchunk = w.nchunk; a.seg_width = w.seg_width;
   a.ids = ids;

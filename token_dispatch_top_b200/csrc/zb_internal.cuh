@@ -59,6 +59,7 @@ inline Workspace workspace_layout(const zb_config& c) {
 struct PlanArgs {
   int P, E, K, S, R, Eh, gpn, cap, policy;
   int relax, cfix;  // eq. (1)'s band: C as floor(C * 2^20), 0 unless relax
+  int repair;       // quota repair between rank pairs after the greedy
   int nchunk, seg_width;
   const int32_t* ids;
   const int32_t* placement;  // [P][R] replica placement to keep, or nullptr

@@ -30,7 +30,7 @@ POLICY_ROOM = 0   # receiver with the most room (after node coverage)
 POLICY_LOCAL = 1  # the largest move, then the most rows served locally
 
 STAT_STATUS, STAT_MAX_LOAD, STAT_N_REPLICAS, STAT_N_ITERS, STAT_WATER_LEVEL, \
-    STAT_LOCALITY_COST, STAT_BAD_IDS = range(7)
+    STAT_LOCALITY_COST, STAT_BAD_IDS, STAT_REPAIRED = range(8)
 STATS_LEN = 8
 
 EXPORTS = ("zb_strerror", "zb_validate", "zb_workspace_bytes", "zb_plan", "zb_plan_placed",
@@ -49,7 +49,7 @@ class _Cfg(ctypes.Structure):
                 ("S", ctypes.c_int), ("H", ctypes.c_int), ("R", ctypes.c_int),
                 ("C", ctypes.c_float), ("gpus_per_node", ctypes.c_int),
                 ("cap_rows", ctypes.c_int), ("policy", ctypes.c_int),
-                ("relax", ctypes.c_int)]
+                ("relax", ctypes.c_int), ("repair", ctypes.c_int)]
 
 
 class _Plan(ctypes.Structure):
@@ -111,6 +111,7 @@ class Config:
     cap_rows: int | None = None  # default S*K, or floor((1+C) S*K) with relax
     policy: int = 0              # POLICY_ROOM or POLICY_LOCAL
     relax: int = 0               # 1: receipts within q +- floor(C q), eq. (1)
+    repair: int = 0              # 1: quota repair between rank pairs
 
     @property
     def cap(self) -> int:
@@ -128,7 +129,7 @@ class Config:
 
     def c(self) -> _Cfg:
         return _Cfg(self.P, self.E, self.K, self.S, self.H, self.R, float(self.C),
-                    self.gpus_per_node, self.cap, self.policy, self.relax)
+                    self.gpus_per_node, self.cap, self.policy, self.relax, self.repair)
 
 
 def validate(cfg: Config) -> int:
