@@ -85,6 +85,10 @@ def _load():
         lib.zbo_merge.restype = None
         lib.zbo_dispatch_merged.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp]
         lib.zbo_dispatch_merged.restype = None
+        lib.zbo_combine_reduce.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, vp, vp]
+        lib.zbo_combine_reduce.restype = None
+        lib.zbo_combine_merged.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp]
+        lib.zbo_combine_merged.restype = None
         d = ctypes.POINTER(ctypes.c_double)
         lib.zbo_metrics.argtypes = [ctypes.POINTER(_Cfg), _P32, _P32, _P32, d, d, d, d]
         lib.zbo_metrics.restype = None
@@ -224,6 +228,33 @@ def dispatch_merged(cfg: Config, tok_row: np.ndarray, hidden_bits: np.ndarray,
     _load().zbo_dispatch_merged(ctypes.byref(cfg.c()), tok_row.ctypes.data,
                                 hidden_bits.ctypes.data, tbuf_bits.ctypes.data)
     return tbuf_bits
+
+
+def combine_reduce(cfg: Config, dst_row: np.ndarray, tok_row: np.ndarray, y_bits: np.ndarray,
+                   w: np.ndarray, part_bits: np.ndarray | None = None) -> np.ndarray:
+    """Destination side of the merged combine: one bf16 partial per merged
+    row, ``part`` uint16 ``[P,cap,H]`` (rows no token names keep their value)."""
+    P, H = cfg.P, cfg.H
+    dst_row = np.ascontiguousarray(dst_row, dtype=np.int32)
+    tok_row = np.ascontiguousarray(tok_row, dtype=np.int32)
+    y_bits = np.ascontiguousarray(y_bits, dtype=np.uint16)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    if part_bits is None:
+        part_bits = np.zeros((P, cfg.cap(), H), np.uint16)
+    _load().zbo_combine_reduce(ctypes.byref(cfg.c()), dst_row.ctypes.data, tok_row.ctypes.data,
+                               y_bits.ctypes.data, w.ctypes.data, part_bits.ctypes.data)
+    return part_bits
+
+
+def combine_merged(cfg: Config, tok_row: np.ndarray, part_bits: np.ndarray) -> np.ndarray:
+    """Source side of the merged combine: ``out`` uint16 ``[P,S,H]``."""
+    P, S, H = cfg.P, cfg.S, cfg.H
+    tok_row = np.ascontiguousarray(tok_row, dtype=np.int32)
+    part_bits = np.ascontiguousarray(part_bits, dtype=np.uint16)
+    out = np.zeros((P, S, H), np.uint16)
+    _load().zbo_combine_merged(ctypes.byref(cfg.c()), tok_row.ctypes.data, part_bits.ctypes.data,
+                               out.ctypes.data)
+    return out
 
 
 def f32_to_bf16(x: float) -> int:

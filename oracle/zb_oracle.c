@@ -686,6 +686,64 @@ void zbo_dispatch_merged(const zbo_config *c, const int32_t *tok_row, const uint
              sizeof(uint16_t) * (size_t)H);
 }
 
+float zbo_bf16_to_f32(uint16_t b);
+uint16_t zbo_f32_to_bf16(float f);
+
+/* Combine with node-local pre-reduction [ZEPP 4.2, Merge: on each rank the
+ * outputs of a token's experts are summed into one partial row before it is
+ * sent back].  Destination side: for each merged row r of token t,
+ *   part[r] = bf16( acc ), acc = +0.0f, then acc = fmaf(w[t,k], y[dst_row[t,k]], acc)
+ *   for k = 0..K-1 with tok_row[t,k] = r,
+ * i.e. the plain combine's fold restricted to the experts that rank served,
+ * rounded once to the payload type (bf16) for the transfer.  Merged rows no
+ * token names are not written. */
+void zbo_combine_reduce(const zbo_config *c, const int32_t *dst_row, const int32_t *tok_row,
+                        const uint16_t *y, const float *w, uint16_t *part) {
+  const int K = c->K;
+  const int64_t H = c->H;
+  float *acc = malloc(sizeof(float) * (size_t)H);
+  for (int64_t t = 0; t < (int64_t)c->P * c->S; t++)
+    for (int k0 = 0; k0 < K; k0++) {
+      int32_t r = tok_row[t * K + k0];
+      int first = 1;
+      for (int k = 0; k < k0; k++)
+        if (tok_row[t * K + k] == r) first = 0;
+      if (!first) continue;
+      for (int64_t h = 0; h < H; h++) acc[h] = 0.0f;
+      for (int k = k0; k < K; k++) {
+        if (tok_row[t * K + k] != r) continue;
+        const uint16_t *yr = y + (int64_t)dst_row[t * K + k] * H;
+        const float wk = w[t * K + k];
+        for (int64_t h = 0; h < H; h++) acc[h] = fmaf(wk, zbo_bf16_to_f32(yr[h]), acc[h]);
+      }
+      for (int64_t h = 0; h < H; h++) part[(int64_t)r * H + h] = zbo_f32_to_bf16(acc[h]);
+    }
+  free(acc);
+}
+
+/* Source side of the merged combine: out[t] = bf16( acc ), acc = +0.0f, then
+ * acc = acc + part[r] for the token's merged rows r in the order of the
+ * first k that names each. */
+void zbo_combine_merged(const zbo_config *c, const int32_t *tok_row, const uint16_t *part,
+                        uint16_t *out) {
+  const int K = c->K;
+  const int64_t H = c->H;
+  float *acc = malloc(sizeof(float) * (size_t)H);
+  for (int64_t t = 0; t < (int64_t)c->P * c->S; t++) {
+    for (int64_t h = 0; h < H; h++) acc[h] = 0.0f;
+    for (int k0 = 0; k0 < K; k0++) {
+      int32_t r = tok_row[t * K + k0];
+      int first = 1;
+      for (int k = 0; k < k0; k++)
+        if (tok_row[t * K + k] == r) first = 0;
+      if (!first) continue;
+      for (int64_t h = 0; h < H; h++) acc[h] = acc[h] + zbo_bf16_to_f32(part[(int64_t)r * H + h]);
+    }
+    for (int64_t h = 0; h < H; h++) out[t * H + h] = zbo_f32_to_bf16(acc[h]);
+  }
+  free(acc);
+}
+
 /* ------------------------------------------------ bf16 (IEEE definition) */
 
 /* bf16 is the upper half of an IEEE binary32: widening is exact. */
