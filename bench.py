@@ -353,7 +353,27 @@ def run_ours(args, wl, rank, world, local_rank):
         m_ms.append(a0.elapsed_time(a1))
         d_ms.append(a1.elapsed_time(a2))
     rows_merged = int(merged.tok_cnt.sum())
-    del tbuf
+    # the merged combine: pre-reduce per (token, rank) into bf16 partials, then
+    # add the partials per token; y = the dispatched rows (identity experts)
+    part = torch.empty_like(buf)
+    out_m = torch.empty((P, S, H), dtype=torch.bfloat16, device=dev)
+    zb.dispatch(plan, hidden, buf)
+    zb.combine_reduce(plan, merged, buf, w, part)
+    zb.combine_merged(plan, merged, part, out_m)
+    torch.cuda.synchronize()
+    cr_ms, cm_ms = [], []
+    for _ in range(max(20, min(args.steps, 100))):
+        flush_l2()
+        a0, a1, a2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        a0.record(stream)
+        zb.combine_reduce(plan, merged, buf, w, part)
+        a1.record(stream)
+        zb.combine_merged(plan, merged, part, out_m)
+        a2.record(stream)
+        a2.synchronize()
+        cr_ms.append(a0.elapsed_time(a1))
+        cm_ms.append(a1.elapsed_time(a2))
+    del tbuf, part, out_m
 
     # ---- the banded plan (eq. (1) with its C band in use), timed apart from
     # the step: the same ids planned with relax = 1 and floor((1+C) S*K) rows
@@ -535,6 +555,15 @@ def run_ours(args, wl, rank, world, local_rank):
             "dispatch_ms": statistics.median(d_ms),
             "dispatch_gbs": (wl.tokens * wl.H * 2 + rows_merged * wl.H * 2 + wl.N * 4)
             / statistics.median(d_ms) / 1e6},
+            "merged_combine": {
+                "what": "Zepp 4.2 merge for combine: a bf16 partial per (token, rank), then "
+                        "the partials added per token; not part of the step",
+                "reduce_ms": statistics.median(cr_ms),
+                "reduce_gbs": (wl.N * (wl.H * 2 + 12) + rows_merged * wl.H * 2)
+                / statistics.median(cr_ms) / 1e6,
+                "combine_ms": statistics.median(cm_ms),
+                "combine_gbs": (rows_merged * wl.H * 2 + wl.N * 4 + wl.tokens * wl.H * 2)
+                / statistics.median(cm_ms) / 1e6},
             "banded_plan": banded, "quota_repair": rep},
         "wall_s": wall,
         "clocks": clocks.summary(),

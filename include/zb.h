@@ -319,6 +319,31 @@ ZB_API int zb_dispatch_merged(const zb_config *cfg, const zb_plan_t *plan,
                               const zb_merge_t *merge, const uint16_t *hidden, uint16_t *tbuf,
                               void *stream);
 
+/* Combine with node-local pre-reduction (Zepp, 4.2 Split and Merge: a rank
+ * sums the outputs of the experts a token selected on it into one partial
+ * before sending it back), in two calls, the destination side and the source
+ * side.  The merged layout `merge` must come from zb_merge of the same plan.
+ *
+ * zb_combine_reduce: y bf16 [P][cap][H] (expert outputs in the plan's
+ * expert-grouped rows), topk_weights fp32 [P][S][K] -> part bf16 [P][cap][H]
+ * (merged rows).  For each merged row r of token t:
+ *   acc = +0.0f; acc = fmaf(w[t,k], y[dst_row[t,k]], acc) for k = 0..K-1
+ *   with tok_row[t,k] = r; part[r] = bf16(acc), rounded to nearest even.
+ * Rows past tok_cnt[j] are not written.
+ *
+ * zb_combine_merged: part -> out bf16 [P][S][H]:
+ *   acc = +0.0f; acc = acc + part[r] for the token's merged rows r in the
+ *   order of the first k naming each; out[t] = bf16(acc).
+ * Where all of a token's experts sit on one rank, out equals zb_combine's
+ * output bit for bit; otherwise each partial adds one bf16 rounding.
+ * Both: y, part and out 16-byte aligned; ZB_OK, ZB_ERR_INVALID or
+ * ZB_ERR_CUDA; nothing is written when the plan's status is an error. */
+ZB_API int zb_combine_reduce(const zb_config *cfg, const zb_plan_t *plan, const zb_merge_t *merge,
+                             const uint16_t *y, const float *topk_weights, uint16_t *part,
+                             void *stream);
+ZB_API int zb_combine_merged(const zb_config *cfg, const zb_plan_t *plan, const zb_merge_t *merge,
+                             const uint16_t *part, uint16_t *out, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

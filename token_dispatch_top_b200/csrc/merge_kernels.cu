@@ -9,7 +9,13 @@
 //                   ballots), giving tok_row, grp_tok and tok_cnt
 //   k_dispatch_merged  one warp per token: read the row once, write it once
 //                   per distinct destination row
+//   k_combine_reduce   destination side of the merged combine: one warp per
+//                   token folds the gated outputs each rank served into one
+//                   bf16 partial per merged row (Zepp 4.2: node-local
+//                   pre-reduction into partial sums before transfer)
+//   k_combine_merged   source side: one warp per token adds its partials
 #include "zb_internal.cuh"
+#include "zb_rows.cuh"
 
 namespace zb {
 namespace {
@@ -152,7 +158,7 @@ __global__ void __launch_bounds__(256) k_dispatch_merged(int ntok, int H, int64_
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int v = v0 + 32 * u;
-      if (v < nv) x[u] = __ldcs(src + v);
+      if (v < nv) x[u] = ld_nc(src + v);
     }
 #pragma unroll
     for (int k = 0; k < K; ++k) {
@@ -161,8 +167,121 @@ __global__ void __launch_bounds__(256) k_dispatch_merged(int ntok, int H, int64_
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int v = v0 + 32 * u;
-        if (v < nv) __stcs(dst + v, x[u]);
+        if (v < nv) st_v4(dst + v, x[u]);
       }
+    }
+  }
+}
+
+// Destination side of the merged combine, one warp per token.  Lanes < K hold
+// the token's grouped rows, gates and merged rows.  For each merged row, led
+// by the lowest k that names it, the gated outputs of the k naming it are
+// folded in k order, acc = fmaf(w_k, y_k, acc) from +0.0f, and rounded once
+// to bf16 into that merged row.
+template <int K, int U>
+__global__ void __launch_bounds__(256) k_combine_reduce(int ntok, int H, int64_t nrows,
+                                                        const int32_t* __restrict__ dst_row,
+                                                        const int32_t* __restrict__ tok_row,
+                                                        const int64_t* __restrict__ stats,
+                                                        const uint4* __restrict__ y,
+                                                        const float* __restrict__ w,
+                                                        uint4* __restrict__ part) {
+  if (stats[ZB_STAT_STATUS] < 0) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t t = int64_t(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (t >= ntok) return;
+  const int nv = H >> 3;
+  const int my_d = lane < K ? __ldg(dst_row + t * K + lane) : 0;
+  const int my_m = lane < K ? __ldg(tok_row + t * K + lane) : -2 - lane;
+  const float my_w = lane < K ? __ldg(w + t * K + lane) : 0.f;
+  const unsigned peers = __match_any_sync(kFull, my_m);
+  const unsigned leads = __ballot_sync(kFull, lane < K && (__ffs(peers) - 1) == lane);
+  int64_t rows[K];
+  int mrow[K];
+  float wk[K];
+  bool ok = true;
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const int r = __shfl_sync(kFull, my_d, k);
+    mrow[k] = __shfl_sync(kFull, my_m, k);
+    wk[k] = __shfl_sync(kFull, my_w, k);
+    ok = ok && r >= 0 && r < nrows && mrow[k] >= 0 && mrow[k] < nrows;
+    rows[k] = int64_t(r) * nv;
+  }
+  if (!ok) return;  // a corrupt plan or layout: write nothing for this token
+  for (int v0 = lane; v0 < nv; v0 += 32 * U) {
+    uint4 x[U][K];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int v = v0 + 32 * u;
+      if (v < nv) {
+#pragma unroll
+        for (int k = 0; k < K; ++k) x[u][k] = ld_nc(y + rows[k] + v);
+      }
+    }
+#pragma unroll
+    for (int k0 = 0; k0 < K; ++k0) {
+      if (!((leads >> k0) & 1u)) continue;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int v = v0 + 32 * u;
+        if (v >= nv) continue;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = k0; k < K; ++k)
+          if (mrow[k] == mrow[k0]) fma8(acc, wk[k], x[u][k]);
+        st_v4(part + int64_t(mrow[k0]) * nv + v, pack_bf16x8(acc));
+      }
+    }
+  }
+}
+
+// Source side of the merged combine, one warp per token: out = bf16 of the
+// float sum of the token's partials, acc = acc + part from +0.0f, in the
+// order of the first k naming each merged row.
+template <int K, int U>
+__global__ void __launch_bounds__(256) k_combine_merged(int ntok, int H, int64_t nrows,
+                                                        const int32_t* __restrict__ tok_row,
+                                                        const int64_t* __restrict__ stats,
+                                                        const uint4* __restrict__ part,
+                                                        uint4* __restrict__ out) {
+  if (stats[ZB_STAT_STATUS] < 0) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t t = int64_t(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (t >= ntok) return;
+  const int nv = H >> 3;
+  const int my_m = lane < K ? __ldg(tok_row + t * K + lane) : -2 - lane;
+  const unsigned peers = __match_any_sync(kFull, my_m);
+  const unsigned leads = __ballot_sync(kFull, lane < K && (__ffs(peers) - 1) == lane);
+  int64_t rows[K];
+  bool ok = true;
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const int m = __shfl_sync(kFull, my_m, k);
+    ok = ok && m >= 0 && m < nrows;
+    rows[k] = int64_t(m) * nv;
+  }
+  if (!ok) return;
+  for (int v0 = lane; v0 < nv; v0 += 32 * U) {
+    uint4 x[U][K];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int v = v0 + 32 * u;
+      if (v < nv) {
+#pragma unroll
+        for (int k = 0; k < K; ++k)
+          if ((leads >> k) & 1u) x[u][k] = ld_nc(part + rows[k] + v);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int v = v0 + 32 * u;
+      if (v >= nv) continue;
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < K; ++k)
+        if ((leads >> k) & 1u) add8(acc, x[u][k]);
+      st_v4(out + t * nv + v, pack_bf16x8(acc));
     }
   }
 }
@@ -178,6 +297,28 @@ cudaError_t dispatch_merged_k(int ntok, int H, int64_t nrows, const int32_t* tok
   return cudaGetLastError();
 }
 
+template <int K>
+cudaError_t combine_reduce_k(int ntok, int H, int64_t nrows, const int32_t* dst_row,
+                             const int32_t* tok_row, const int64_t* stats, const uint16_t* y,
+                             const float* w, uint16_t* part, cudaStream_t s) {
+  constexpr int U = K <= 6 ? 4 : (K <= 8 ? 2 : 1);
+  k_combine_reduce<K, U><<<(ntok + 7) / 8, 256, 0, s>>>(
+      ntok, H, nrows, dst_row, tok_row, stats, reinterpret_cast<const uint4*>(y), w,
+      reinterpret_cast<uint4*>(part));
+  return cudaGetLastError();
+}
+
+template <int K>
+cudaError_t combine_merged_k(int ntok, int H, int64_t nrows, const int32_t* tok_row,
+                             const int64_t* stats, const uint16_t* part, uint16_t* out,
+                             cudaStream_t s) {
+  constexpr int U = K <= 6 ? 4 : (K <= 8 ? 2 : 1);
+  k_combine_merged<K, U><<<(ntok + 7) / 8, 256, 0, s>>>(
+      ntok, H, nrows, tok_row, stats, reinterpret_cast<const uint4*>(part),
+      reinterpret_cast<uint4*>(out));
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s) {
@@ -190,9 +331,6 @@ cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-#define ZB_K_CASES(X) \
-  X(1) X(2) X(3) X(4) X(5) X(6) X(7) X(8) X(9) X(10) X(11) X(12) X(13) X(14) X(15) X(16)
-
 cudaError_t launch_dispatch_merged(int P, int S, int K, int H, int cap, const int32_t* tok_row,
                                    const int64_t* stats, const uint16_t* hidden, uint16_t* tbuf,
                                    cudaStream_t s) {
@@ -203,6 +341,41 @@ cudaError_t launch_dispatch_merged(int P, int S, int K, int H, int cap, const in
 #define X(k) \
   case k:    \
     return dispatch_merged_k<k>(ntok, H, nrows, tok_row, stats, hidden, tbuf, s);
+    ZB_K_CASES(X)
+#undef X
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_combine_reduce(int P, int S, int K, int H, int cap, const int32_t* dst_row,
+                                  const int32_t* tok_row, const int64_t* stats,
+                                  const uint16_t* y, const float* w, uint16_t* part,
+                                  cudaStream_t s) {
+  const int ntok = P * S;
+  if (ntok == 0) return cudaSuccess;
+  const int64_t nrows = int64_t(P) * cap;
+  switch (K) {
+#define X(k) \
+  case k:    \
+    return combine_reduce_k<k>(ntok, H, nrows, dst_row, tok_row, stats, y, w, part, s);
+    ZB_K_CASES(X)
+#undef X
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_combine_merged(int P, int S, int K, int H, int cap, const int32_t* tok_row,
+                                  const int64_t* stats, const uint16_t* part, uint16_t* out,
+                                  cudaStream_t s) {
+  const int ntok = P * S;
+  if (ntok == 0) return cudaSuccess;
+  const int64_t nrows = int64_t(P) * cap;
+  switch (K) {
+#define X(k) \
+  case k:    \
+    return combine_merged_k<k>(ntok, H, nrows, tok_row, stats, part, out, s);
     ZB_K_CASES(X)
 #undef X
     default:

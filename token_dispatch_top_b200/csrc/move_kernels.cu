@@ -7,20 +7,14 @@
 // Sources: MoonEP "What MoonEP enforces and how" (zero-copy writes into
 // fixed-shape expert-grouped buffers); Zepp "4.2 Split and Merge" (combine);
 // ISER-MoE "Key Formula" (dispatch + combine traffic term).
-#include <cuda_bf16.h>
-
 #include "zb_internal.cuh"
+#include "zb_rows.cuh"
 
 namespace zb {
 namespace {
 
 constexpr int kMoveThreads = 256;
 constexpr int kMoveWarps = kMoveThreads / 32;
-
-// Every row is read once and written once per destination: streaming
-// (evict-first) loads and stores keep the 126 MB L2 for the small plan tables.
-__device__ __forceinline__ uint4 ld_nc(const uint4* p) { return __ldcs(p); }
-__device__ __forceinline__ void st_v4(uint4* p, const uint4& v) { __stcs(p, v); }
 
 // One warp per token t = i*S + s: read the row once, write it to its K rows.
 template <int K, int U>
@@ -60,27 +54,6 @@ __global__ void __launch_bounds__(kMoveThreads) k_dispatch(int ntok, int H, int6
       }
     }
   }
-}
-
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
-  const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
-  return l | (h << 16);
-}
-
-// acc = fmaf(w, y, acc) on the 8 bf16 lanes of one 16-byte vector.
-__device__ __forceinline__ void fma8(float (&acc)[8], float w, const uint4& y) {
-  acc[0] = __fmaf_rn(w, bf_lo(y.x), acc[0]);
-  acc[1] = __fmaf_rn(w, bf_hi(y.x), acc[1]);
-  acc[2] = __fmaf_rn(w, bf_lo(y.y), acc[2]);
-  acc[3] = __fmaf_rn(w, bf_hi(y.y), acc[3]);
-  acc[4] = __fmaf_rn(w, bf_lo(y.z), acc[4]);
-  acc[5] = __fmaf_rn(w, bf_hi(y.z), acc[5]);
-  acc[6] = __fmaf_rn(w, bf_lo(y.w), acc[6]);
-  acc[7] = __fmaf_rn(w, bf_hi(y.w), acc[7]);
 }
 
 // One warp per token: gather its K rows, fold them with one fused
@@ -127,12 +100,7 @@ __global__ void __launch_bounds__(kMoveThreads) k_combine(int ntok, int H, int64
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int k = 0; k < K; ++k) fma8(acc, wk[k], x[u][k]);
-        uint4 o;
-        o.x = pack_bf16x2(acc[0], acc[1]);
-        o.y = pack_bf16x2(acc[2], acc[3]);
-        o.z = pack_bf16x2(acc[4], acc[5]);
-        o.w = pack_bf16x2(acc[6], acc[7]);
-        st_v4(out + t * nv + v, o);
+        st_v4(out + t * nv + v, pack_bf16x8(acc));
       }
     }
   }
@@ -162,9 +130,6 @@ cudaError_t combine_k(int ntok, int H, int64_t nrows, const int32_t* dst_row,
 }
 
 }  // namespace
-
-#define ZB_K_CASES(X) \
-  X(1) X(2) X(3) X(4) X(5) X(6) X(7) X(8) X(9) X(10) X(11) X(12) X(13) X(14) X(15) X(16)
 
 cudaError_t launch_dispatch(int P, int S, int K, int H, int cap, const int32_t* dst_row,
                             const int64_t* stats, const uint16_t* hidden, uint16_t* buf,

@@ -189,6 +189,28 @@ int zb_dispatch_merged(const zb_config* c, const zb_plan_t* plan, const zb_merge
   return ZB_OK;
 }
 
+int zb_combine_reduce(const zb_config* c, const zb_plan_t* plan, const zb_merge_t* m,
+                      const uint16_t* y, const float* w, uint16_t* part, void* stream) {
+  if (zb_validate(c) != ZB_OK || !plan || !plan->stats || !m) return ZB_ERR_INVALID;
+  if (c->S > 0 && (!plan->dst_row || !m->tok_row || !y || !w || !part)) return ZB_ERR_INVALID;
+  if ((y && !aligned16(y)) || (part && !aligned16(part))) return ZB_ERR_INVALID;
+  if (zb::launch_combine_reduce(c->P, c->S, c->K, c->H, c->cap_rows, plan->dst_row, m->tok_row,
+                                plan->stats, y, w, part, as_stream(stream)) != cudaSuccess)
+    return ZB_ERR_CUDA;
+  return ZB_OK;
+}
+
+int zb_combine_merged(const zb_config* c, const zb_plan_t* plan, const zb_merge_t* m,
+                      const uint16_t* part, uint16_t* out, void* stream) {
+  if (zb_validate(c) != ZB_OK || !plan || !plan->stats || !m) return ZB_ERR_INVALID;
+  if (c->S > 0 && (!m->tok_row || !part || !out)) return ZB_ERR_INVALID;
+  if ((part && !aligned16(part)) || (out && !aligned16(out))) return ZB_ERR_INVALID;
+  if (zb::launch_combine_merged(c->P, c->S, c->K, c->H, c->cap_rows, m->tok_row, plan->stats,
+                                part, out, as_stream(stream)) != cudaSuccess)
+    return ZB_ERR_CUDA;
+  return ZB_OK;
+}
+
 int zb_combine(const zb_config* c, const zb_plan_t* plan, const uint16_t* y, const float* w,
                uint16_t* out, void* stream) {
   if (zb_validate(c) != ZB_OK || !plan || !plan->stats) return ZB_ERR_INVALID;

@@ -106,6 +106,13 @@ cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s);
 cudaError_t launch_dispatch_merged(int P, int S, int K, int H, int cap, const int32_t* tok_row,
                                    const int64_t* stats, const uint16_t* hidden, uint16_t* tbuf,
                                    cudaStream_t s);
+cudaError_t launch_combine_reduce(int P, int S, int K, int H, int cap, const int32_t* dst_row,
+                                  const int32_t* tok_row, const int64_t* stats,
+                                  const uint16_t* y, const float* w, uint16_t* part,
+                                  cudaStream_t s);
+cudaError_t launch_combine_merged(int P, int S, int K, int H, int cap, const int32_t* tok_row,
+                                  const int64_t* stats, const uint16_t* part, uint16_t* out,
+                                  cudaStream_t s);
 cudaError_t launch_combine(int P, int S, int K, int H, int cap, const int32_t* dst_row,
                            const int64_t* stats, const uint16_t* y, const float* w,
                            uint16_t* out, cudaStream_t s);

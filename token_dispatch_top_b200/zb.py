@@ -35,7 +35,7 @@ STATS_LEN = 8
 
 EXPORTS = ("zb_strerror", "zb_validate", "zb_workspace_bytes", "zb_plan", "zb_plan_placed",
            "zb_plan_status", "zb_dispatch", "zb_combine", "zb_merge_workspace_bytes",
-           "zb_merge", "zb_dispatch_merged")
+           "zb_merge", "zb_dispatch_merged", "zb_combine_reduce", "zb_combine_merged")
 
 
 class ZbError(RuntimeError):
@@ -89,6 +89,8 @@ def load() -> ctypes.CDLL:
         lib.zb_merge_workspace_bytes.restype = ctypes.c_size_t
         lib.zb_merge.argtypes = [cfgp, planp, mergep, vp, ctypes.c_size_t, vp]
         lib.zb_dispatch_merged.argtypes = [cfgp, planp, mergep, vp, vp, vp]
+        lib.zb_combine_reduce.argtypes = [cfgp, planp, mergep, vp, vp, vp, vp]
+        lib.zb_combine_merged.argtypes = [cfgp, planp, mergep, vp, vp, vp]
         _lib = lib
     return _lib
 
@@ -279,3 +281,32 @@ def dispatch_merged(p: Plan, m: Merge, hidden: torch.Tensor, tbuf: torch.Tensor,
                                    hidden.data_ptr(), tbuf.data_ptr(), _stream(stream))
     if st != OK:
         raise ZbError(st, "zb_dispatch_merged")
+
+
+def combine_reduce(p: Plan, m: Merge, y: torch.Tensor, topk_weights: torch.Tensor,
+                   part: torch.Tensor, stream=None) -> None:
+    """Destination side of the merged combine: ``y`` bf16 [P,cap,H] (expert
+    outputs in grouped rows), ``topk_weights`` fp32 [P,S,K] -> ``part`` bf16
+    [P,cap,H], one partial per merged row (rows past m.tok_cnt untouched)."""
+    cfg = p.cfg
+    _check(y, (cfg.P, cfg.cap, cfg.H), torch.bfloat16, "y")
+    _check(topk_weights, (cfg.P, cfg.S, cfg.K), torch.float32, "topk_weights")
+    _check(part, (cfg.P, cfg.cap, cfg.H), torch.bfloat16, "part")
+    st = load().zb_combine_reduce(ctypes.byref(p._c), ctypes.byref(p._p), ctypes.byref(m._m),
+                                  y.data_ptr(), topk_weights.data_ptr(), part.data_ptr(),
+                                  _stream(stream))
+    if st != OK:
+        raise ZbError(st, "zb_combine_reduce")
+
+
+def combine_merged(p: Plan, m: Merge, part: torch.Tensor, out: torch.Tensor,
+                   stream=None) -> None:
+    """Source side of the merged combine: ``part`` bf16 [P,cap,H] -> ``out``
+    bf16 [P,S,H], the float sum of each token's partials rounded once."""
+    cfg = p.cfg
+    _check(part, (cfg.P, cfg.cap, cfg.H), torch.bfloat16, "part")
+    _check(out, (cfg.P, cfg.S, cfg.H), torch.bfloat16, "out")
+    st = load().zb_combine_merged(ctypes.byref(p._c), ctypes.byref(p._p), ctypes.byref(m._m),
+                                  part.data_ptr(), out.data_ptr(), _stream(stream))
+    if st != OK:
+        raise ZbError(st, "zb_combine_merged")
