@@ -85,6 +85,9 @@ def _load():
         lib.zbo_merge.restype = None
         lib.zbo_dispatch_merged.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp]
         lib.zbo_dispatch_merged.restype = None
+        lib.zbo_recalibrate.argtypes = [ctypes.POINTER(_Cfg), _P32, _P32, ctypes.c_int,
+                                        ctypes.c_double, ctypes.c_int, _P32]
+        lib.zbo_recalibrate.restype = ctypes.c_int
         lib.zbo_combine_reduce.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, vp, vp]
         lib.zbo_combine_reduce.restype = None
         lib.zbo_combine_merged.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp]
@@ -228,6 +231,20 @@ def dispatch_merged(cfg: Config, tok_row: np.ndarray, hidden_bits: np.ndarray,
     _load().zbo_dispatch_merged(ctypes.byref(cfg.c()), tok_row.ctypes.data,
                                 hidden_bits.ctypes.data, tbuf_bits.ctypes.data)
     return tbuf_bits
+
+
+def recalibrate(cfg: Config, cnt: np.ndarray, placement: np.ndarray, mode: int, eps: float,
+                max_swaps: int) -> tuple[np.ndarray, int, int]:
+    """Placement recalibration (mode 0: one slot changed per step; mode 1:
+    intra-node slot swaps).  Returns (new placement, steps, final max load)."""
+    cnt = np.ascontiguousarray(cnt, dtype=np.int32).reshape(cfg.P, cfg.E)
+    pl = np.ascontiguousarray(placement, dtype=np.int32).reshape(cfg.P, cfg.R).copy()
+    mx = np.zeros(1, np.int32)
+    n = _load().zbo_recalibrate(ctypes.byref(cfg.c()), _ptr(cnt), _ptr(pl), int(mode),
+                                float(eps), int(max_swaps), _ptr(mx))
+    if n < 0:
+        raise ValueError(f"zbo_recalibrate: status {n}")
+    return pl, int(n), int(mx[0])
 
 
 def combine_reduce(cfg: Config, dst_row: np.ndarray, tok_row: np.ndarray, y_bits: np.ndarray,

@@ -643,6 +643,111 @@ int zbo_plan_placed(const zbo_config *c, const int32_t *ids, const int32_t *plac
   return status;
 }
 
+/* ------------------------------------------ placement recalibration */
+
+/* Max rank load of the kept-placement plan (greedy_placed over `placement`)
+ * for route counts cnt: what both searches below minimise.  Scratch: rq, hq
+ * [E], load [P]. */
+static int32_t placed_max_load(const zbo_config *c, const int32_t *cnt, const int32_t *placement,
+                               int32_t *rq, int32_t *hq, int32_t *load) {
+  const int P = c->P, E = c->E, Eh = E / P;
+  int64_t sum = 0;
+  for (int e = 0; e < E; e++) {
+    hq[e] = 0;
+    for (int i = 0; i < P; i++) hq[e] += cnt[(size_t)i * E + e];
+  }
+  for (int j = 0; j < P; j++) {
+    load[j] = 0;
+    for (int e = j * Eh; e < (j + 1) * Eh; e++) load[j] += hq[e];
+    sum += load[j];
+  }
+  int32_t T = (int32_t)((sum + P - 1) / P), iters, mx = 0;
+  greedy_placed(c, T, load, hq, placement, rq, &iters);
+  for (int j = 0; j < P; j++)
+    if (load[j] > mx) mx = load[j];
+  return mx;
+}
+
+/* Whether helper slot s of rank r may hold expert e: e is homed elsewhere
+ * and no other slot of r holds it. */
+static int slot_takes(const zbo_config *c, const int32_t *pl, int r, int s, int e) {
+  if (e / (c->E / c->P) == r) return 0;
+  for (int t = 0; t < c->R; t++)
+    if (t != s && pl[r * c->R + t] == e) return 0;
+  return 1;
+}
+
+/* Placement recalibration between invocations, on the route counts cnt of
+ * the invocation that triggered it.  Candidates, in enumeration order:
+ *  mode 0 [ViBE, Drift-Aware Recalibration, incremental placement update:
+ *    start from the current placement, apply minimal cross-GPU expert swaps]:
+ *    helper slot x ascending, then expert e ascending: slot x now holds e
+ *    (a copy of e moves in, one weight transfer);
+ *  mode 1 [Zepp 4.3, eq. (4): intra-node swaps that exchange expert replicas
+ *    between GPUs of one node, keeping the node's coverage]: slot pairs
+ *    x1 < x2 on two ranks of one node, exchanging their experts (one may be
+ *    empty, moving the other).
+ * Each step takes the candidate whose kept-placement plan has the lowest max
+ * load, the first in order among equals, and only if that is below the
+ * current max load.  The search stops when max load <= (1 + eps) * sum L / P
+ * (every rank within eps of the mean; eps as float), when no candidate lowers
+ * the max load, or after max_swaps steps.  Returns the steps taken; the
+ * final max load goes to *max_load. */
+int zbo_recalibrate(const zbo_config *c, const int32_t *cnt, int32_t *placement, int mode,
+                    double eps, int max_swaps, int32_t *max_load) {
+  if (zbo_validate(c) || !zbo_placement_valid(c, placement)) return ZBO_ERR_INVALID;
+  const int P = c->P, E = c->E, R = c->R, n = P * R;
+  int32_t *rq = malloc(sizeof(int32_t) * (size_t)(n > 0 ? n : 1));
+  int32_t *hq = malloc(sizeof(int32_t) * (size_t)E), *load = malloc(sizeof(int32_t) * (size_t)P);
+  int64_t sum = 0;
+  for (int64_t x = 0; x < (int64_t)P * E; x++) sum += cnt[x];
+  const double bound = (1.0 + (double)(float)eps) * (double)sum / (double)P;
+  int32_t cur = placed_max_load(c, cnt, placement, rq, hq, load);
+  int swaps = 0;
+  while (swaps < max_swaps && (double)cur > bound) {
+    int32_t best = cur;
+    int bx1 = -1, bx2 = -1, be = -1;
+    if (mode == 0) {
+      for (int x = 0; x < n; x++)
+        for (int e = 0; e < E; e++) {
+          int old = placement[x];
+          if (e == old || !slot_takes(c, placement, x / R, x % R, e)) continue;
+          placement[x] = e;
+          int32_t m = placed_max_load(c, cnt, placement, rq, hq, load);
+          placement[x] = old;
+          if (m < best) { best = m; bx1 = x; be = e; }
+        }
+    } else {
+      for (int x1 = 0; x1 < n; x1++)
+        for (int x2 = x1 + 1; x2 < n; x2++) {
+          int r1 = x1 / R, r2 = x2 / R, e1 = placement[x1], e2 = placement[x2];
+          if (r1 == r2 || node_of(c, r1) != node_of(c, r2) || e1 == e2) continue;
+          if (e2 >= 0 && !slot_takes(c, placement, r1, x1 % R, e2)) continue;
+          if (e1 >= 0 && !slot_takes(c, placement, r2, x2 % R, e1)) continue;
+          placement[x1] = e2;
+          placement[x2] = e1;
+          int32_t m = placed_max_load(c, cnt, placement, rq, hq, load);
+          placement[x1] = e1;
+          placement[x2] = e2;
+          if (m < best) { best = m; bx1 = x1; bx2 = x2; }
+        }
+    }
+    if (bx1 < 0) break;
+    if (mode == 0) {
+      placement[bx1] = be;
+    } else {
+      int t = placement[bx1];
+      placement[bx1] = placement[bx2];
+      placement[bx2] = t;
+    }
+    cur = best;
+    swaps++;
+  }
+  if (max_load) *max_load = cur;
+  free(rq); free(hq); free(load);
+  return swaps;
+}
+
 /* ------------------------------------- merged dispatch (Zepp 4.2, merge) */
 
 /* One row per (token, destination rank) instead of one per (token, k): when
