@@ -344,6 +344,34 @@ ZB_API int zb_combine_reduce(const zb_config *cfg, const zb_plan_t *plan, const 
 ZB_API int zb_combine_merged(const zb_config *cfg, const zb_plan_t *plan, const zb_merge_t *merge,
                              const uint16_t *part, uint16_t *out, void *stream);
 
+/* Placement recalibration between invocations (not part of an invocation's
+ * path).  From the replica placement `placement` (device int32 [P][R], -1 =
+ * empty; changed in place) and the route counts `cnt` (device int32 [P][E],
+ * e.g. plan->cnt of the invocation that showed drift), each step applies the
+ * candidate whose kept-placement plan (zb_plan_placed's quotas) has the
+ * lowest max rank load, the first in candidate order among equals, and only
+ * if it lowers the max load.  The search stops once
+ *   max load <= (1 + eps) * (sum of cnt) / P
+ * (every rank within eps of the mean; ViBE's default eps is 0.03), when no
+ * candidate lowers the max load, or after max_swaps steps.
+ *   mode 0 (ViBE, Drift-Aware Recalibration, incremental placement update):
+ *     a candidate puts expert e into helper slot x (one copy moved in over
+ *     the network); order: x = j*R + slot ascending, then e ascending.
+ *   mode 1 (Zepp, 4.3, eq. (4), intra-node swaps): a candidate exchanges the
+ *     experts of slots x1 < x2 on two ranks of one node (one may be empty),
+ *     keeping the node's set of experts; order: x1, then x2 ascending.
+ * A candidate must leave a valid placement (see zb_plan_placed).  Every step
+ * scores all candidates on the device, one warp each, and reads the scores
+ * back: this call synchronises `stream`.  workspace:
+ * zb_recalibrate_workspace_bytes(cfg, mode) bytes, 256-byte aligned.  On
+ * ZB_OK, *swaps (steps taken) and *max_load (the final plan's max rank load)
+ * are written when non-NULL.  ZB_ERR_INVALID for a bad argument, an invalid
+ * placement or negative counts; ZB_ERR_CUDA if a CUDA call fails. */
+ZB_API size_t zb_recalibrate_workspace_bytes(const zb_config *cfg, int mode);
+ZB_API int zb_recalibrate(const zb_config *cfg, const int32_t *cnt, int32_t *placement, int mode,
+                          float eps, int max_swaps, void *workspace, size_t workspace_bytes,
+                          void *stream, int32_t *swaps, int32_t *max_load);
+
 #ifdef __cplusplus
 }
 #endif

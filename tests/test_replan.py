@@ -49,7 +49,16 @@ def test_replanner_plans_match_oracle(cuda_device, strategy):
         w = np.bincount(ids.ravel(), minlength=wl.E)
         if rep.drift is not None:
             assert rep.drift == pytest.approx(replan.cosine_drift(w, w_ref_before), abs=1e-12)
-        if rep.replaced:
+        if strategy == "incremental" and t > 0:
+            # recalibrated from the kept placement when drift or capacity asks
+            kept = oracle.plan(oc, ids, want_M=False, placement=placement)
+            if rep.drift > 0.01 or kept["status"] == oracle.ERR_CAPACITY:
+                placement = oracle.recalibrate(oc, kept["cnt"], placement, 0, 0.03, 64)[0]
+                o = oracle.plan(oc, ids, want_M=False, placement=placement)
+            else:
+                o = kept
+            replaced_later += rep.replaced
+        elif rep.replaced:
             o = oracle.plan(oc, ids, want_M=False)
             placement = o["rep_expert"]
             replaced_later += t > 0
@@ -60,5 +69,7 @@ def test_replanner_plans_match_oracle(cuda_device, strategy):
         assert replaced_later == 0
     elif strategy == "every":
         assert replaced_later == 11
+    elif strategy == "incremental":
+        assert replaced_later > 0
     else:
         assert 0 < replaced_later < 11

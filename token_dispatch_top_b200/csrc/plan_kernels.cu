@@ -242,8 +242,9 @@ __device__ void greedy_warp(const PlanArgs& a, PlannerSmem& s, int T, int load, 
 // or exhausts the expert's home quota: at most 3P + E iterations with the
 // stuck marks.  (Zepp 4.1: replicas placed from historical demand; ViBE:
 // placement recalibrated only on drift.)
-__device__ void greedy_placed_warp(const PlanArgs& a, PlannerSmem& s, int T, int load,
-                                   int lane) {
+// Returns this lane's rank load after the moves (lanes >= P: 0).
+__device__ int greedy_placed_warp(const PlanArgs& a, PlannerSmem& s, int T, int load,
+                                  int lane) {
   const int P = a.P, R = a.R, Eh = a.Eh;
   bool stuck = lane >= P;
   int iters = 0;
@@ -295,7 +296,6 @@ __device__ void greedy_placed_warp(const PlanArgs& a, PlannerSmem& s, int T, int
   int nrep = 0;
   if (lane < P)
     for (int sl = 0; sl < R; ++sl) nrep += s.repe[lane * R + sl] >= 0;
-  if (lane < P) a.load_after[lane] = load;
   const int mx = int(__reduce_max_sync(kFull, lane < P ? unsigned(load) : 0u));
   nrep = int(__reduce_add_sync(kFull, unsigned(nrep)));
   if (lane == 0) {
@@ -303,6 +303,7 @@ __device__ void greedy_placed_warp(const PlanArgs& a, PlannerSmem& s, int T, int
     s.misc[kMiscNrep] = nrep;
     s.misc[kMiscIters] = iters;
   }
+  return lane < P ? load : 0;
 }
 
 // Quota of the copy at quota index x (x < E: home quota of x; else helper
@@ -668,9 +669,10 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
     const long long total = warp_sum64(lane < P ? (long long)L : 0ll);
     const int T = int((total + P - 1) / P);
     if (lane == 0) s.misc[kMiscT] = T;
-    if (kMode == 2)
-      greedy_placed_warp(a, s, T, L, lane);
-    else
+    if (kMode == 2) {
+      const int load = greedy_placed_warp(a, s, T, L, lane);
+      if (lane < P) a.load_after[lane] = load;
+    } else
       greedy_warp<kMode>(a, s, T, L, lane);
   }
   __syncthreads();
@@ -877,6 +879,86 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
   }
 }
 
+// ------------------------------------------------ placement recalibration
+
+// Candidate placements scored by the kept-placement greedy, one warp each:
+// candidate 0 is the base placement; in mode 0 candidate 1 + x*E + e puts
+// expert e into helper slot x; in mode 1 candidate 1 + x1*(P*R) + x2 (x1 <
+// x2, ranks of one node) exchanges the experts of slots x1 and x2.  An
+// invalid candidate scores INT32_MAX.  The score is the plan's max rank load
+// (ViBE, Drift-Aware Recalibration; Zepp 4.3, eq. (4)).
+__global__ void __launch_bounds__(kEvalThreads) k_eval_placements(EvalArgs ea) {
+  extern __shared__ __align__(16) char smem_raw[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t c = int64_t(blockIdx.x) * kEvalWarps + warp;
+  if (c >= ea.ncand) return;
+  const int P = ea.P, E = ea.E, R = ea.R, Eh = E / P, n = P * R, gpn = ea.gpn;
+  const int words = 2 * E + 2 * n + 16;
+  int32_t* base = reinterpret_cast<int32_t*>(smem_raw) + warp * words;
+  PlannerSmem s{};
+  s.hq = base;
+  s.hold = reinterpret_cast<uint32_t*>(base + E);
+  s.repe = base + 2 * E;
+  s.repq = base + 2 * E + n;
+  s.misc = base + 2 * E + 2 * n;
+  // the candidate's change: slot xa gets ea_e (and slot xb gets eb_e)
+  int xa = -1, xb = -1, ea_e = -1, eb_e = -1;
+  bool ok = true;
+  if (c > 0) {
+    const int64_t k = c - 1;
+    if (ea.mode == 0) {
+      xa = int(k / E);
+      ea_e = int(k - int64_t(xa) * E);
+      ok = ea_e != ea.base[xa];
+    } else {
+      xa = int(k / n);
+      xb = int(k - int64_t(xa) * n);
+      ea_e = ea.base[xb];
+      eb_e = ea.base[xa];
+      const int ra = xa / R, rb = xb / R;
+      ok = xa < xb && ra != rb && ra / gpn == rb / gpn && ea_e != eb_e;
+    }
+  }
+  for (int x = lane; x < n; x += 32) {
+    s.repe[x] = x == xa ? ea_e : (x == xb ? eb_e : ea.base[x]);
+    s.repq[x] = 0;
+  }
+  __syncwarp();
+  // a changed slot may hold its expert only if the expert is homed elsewhere
+  // and no other slot of that rank holds it
+  auto takes = [&](int x) {
+    const int e = s.repe[x];
+    if (e < 0) return true;
+    const int r = x / R;
+    if (e / Eh == r) return false;
+    for (int t = r * R; t < r * R + R; ++t)
+      if (t != x && s.repe[t] == e) return false;
+    return true;
+  };
+  if (ok && c > 0) ok = takes(xa) && (xb < 0 || takes(xb));
+  if (!ok) {
+    if (lane == 0) ea.out[c] = INT32_MAX;
+    return;
+  }
+  for (int e = lane; e < E; e += 32) {
+    s.hq[e] = ea.Te[e];
+    s.hold[e] = 0u;
+  }
+  __syncwarp();
+  for (int x = lane; x < n; x += 32)
+    if (s.repe[x] >= 0) atomicOr(&s.hold[s.repe[x]], 1u << (x / R));
+  __syncwarp();
+  int L = 0;
+  if (lane < P)
+    for (int e = lane * Eh; e < (lane + 1) * Eh; ++e) L += s.hq[e];
+  const long long total = warp_sum64(lane < P ? (long long)L : 0ll);
+  const int T = int((total + P - 1) / P);
+  PlanArgs a{};
+  a.P = P; a.E = E; a.R = R; a.Eh = Eh;
+  greedy_placed_warp(a, s, T, L, lane);
+  if (lane == 0) ea.out[c] = s.misc[kMiscMax];
+}
+
 }  // namespace
 
 size_t planner_smem_bytes(const zb_config& c) {
@@ -927,6 +1009,29 @@ cudaError_t launch_planner(const PlanArgs& a, size_t smem, cudaStream_t s) {
                    : launch_planner_variant<true, false>(a, smem, s);
   return a.relax ? launch_planner_variant<false, true>(a, smem, s)
                  : launch_planner_variant<false, false>(a, smem, s);
+}
+
+size_t eval_smem_bytes(int P, int E, int R) {
+  return size_t(kEvalWarps) * size_t(2 * E + 2 * P * R + 16) * sizeof(int32_t);
+}
+
+cudaError_t launch_eval_placements(const EvalArgs& ea, cudaStream_t s) {
+  if (ea.ncand == 0) return cudaSuccess;
+  const size_t smem = eval_smem_bytes(ea.P, ea.E, ea.R);
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    err = cudaFuncSetAttribute(k_eval_placements, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               200 * 1024);
+    if (err != cudaSuccess) return err;
+    configured[dev] = true;
+  }
+  const int64_t blocks = (ea.ncand + kEvalWarps - 1) / kEvalWarps;
+  k_eval_placements<<<unsigned(blocks), kEvalThreads, smem, s>>>(ea);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_assign(const PlanArgs& a, cudaStream_t s) {

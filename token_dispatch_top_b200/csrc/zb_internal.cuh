@@ -78,6 +78,18 @@ struct PlanArgs {
   int2* seg;
 };
 
+// Candidate placements scored by the kept-placement greedy (recalibration).
+constexpr int kEvalThreads = 256;
+constexpr int kEvalWarps = kEvalThreads / 32;
+
+struct EvalArgs {
+  int P, E, R, gpn, mode;
+  int64_t ncand;           // candidate 0 is the base placement
+  const int32_t* Te;       // [E] rows per expert
+  const int32_t* base;     // [P*R] the placement candidates change
+  int32_t* out;            // [ncand] max rank load, INT32_MAX when invalid
+};
+
 // Tokens per CTA of the merged-dispatch layout kernels.
 constexpr int kMergeChunk = 256;
 
@@ -98,6 +110,8 @@ size_t planner_smem_bytes(const zb_config& c);
 cudaError_t launch_hist(const PlanArgs& a, cudaStream_t s);
 cudaError_t launch_planner(const PlanArgs& a, size_t smem, cudaStream_t s);
 cudaError_t launch_assign(const PlanArgs& a, cudaStream_t s);
+size_t eval_smem_bytes(int P, int E, int R);
+cudaError_t launch_eval_placements(const EvalArgs& ea, cudaStream_t s);
 
 cudaError_t launch_dispatch(int P, int S, int K, int H, int cap, const int32_t* dst_row,
                             const int64_t* stats, const uint16_t* hidden, uint16_t* buf,

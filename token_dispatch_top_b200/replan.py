@@ -15,7 +15,11 @@ pages weigh this three ways:
   re-place when the cosine distance d = 1 - w.w_ref / (|w| |w_ref|) between
   this invocation's per-expert load w and the load the placement was made for
   exceeds delta (ViBE, drift detection, delta = 0.05), or when the kept
-  placement no longer fits the receive buffers.
+  placement no longer fits the receive buffers;
+* ``incremental`` - the same trigger, but instead of a fresh placement the
+  kept one is recalibrated (ViBE's incremental update, zb_recalibrate mode
+  0): one helper slot changes per step until every rank is within eps = 0.03
+  of the mean or no change helps, so only the changed slots move weights.
 
 Every invocation is planned on the GPU (zb_plan for a new placement,
 zb_plan_placed to keep one); the drift decision reads the invocation's
@@ -34,7 +38,7 @@ import torch
 
 from . import zb
 
-STRATEGIES = ("every", "static", "drift")
+STRATEGIES = ("every", "static", "drift", "incremental")
 
 
 def cosine_drift(w: np.ndarray, w_ref: np.ndarray) -> float:
@@ -64,7 +68,7 @@ def decide(strategy: str, have_placement: bool, drift: float | None, delta: floa
         return True
     if strategy == "static":
         return False
-    return drift is not None and drift > delta
+    return drift is not None and drift > delta  # drift and incremental
 
 
 @dataclass
@@ -80,10 +84,12 @@ class StepReport:
 class Replanner:
     """Plans a stream of invocations of one shape under a placement policy."""
 
-    def __init__(self, cfg: zb.Config, device, strategy: str = "drift", delta: float = 0.05):
+    def __init__(self, cfg: zb.Config, device, strategy: str = "drift", delta: float = 0.05,
+                 eps: float = 0.03, max_swaps: int = 64):
         if strategy not in STRATEGIES:
             raise ValueError(f"unknown strategy {strategy!r}")
         self.cfg, self.strategy, self.delta = cfg, strategy, delta
+        self.eps, self.max_swaps = eps, max_swaps
         self.plan = zb.Plan(cfg, device, with_row_src=False)
         self.placement: torch.Tensor | None = None
         self.w_ref: np.ndarray | None = None
@@ -106,12 +112,19 @@ class Replanner:
             zb.plan_placed(self.plan, ids, self.placement)
             status, _ = zb.plan_status(self.plan)
             w = self.plan.cnt.sum(0).cpu().numpy()
-            if self.strategy == "drift":
+            if self.strategy in ("drift", "incremental"):
                 drift = cosine_drift(w, self.w_ref)
             replaced, changes = False, 0
             # a kept placement that no longer fits the buffers forces a new one
-            forced = self.strategy == "drift" and status == zb.ERR_CAPACITY
-            if forced or decide(self.strategy, True, drift, self.delta):
+            forced = self.strategy in ("drift", "incremental") and status == zb.ERR_CAPACITY
+            if self.strategy == "incremental" and (forced or decide(self.strategy, True, drift,
+                                                                    self.delta)):
+                changes, _ = zb.recalibrate(self.cfg, self.plan.cnt, self.placement,
+                                            zb.RECAL_SLOT, self.eps, self.max_swaps)
+                zb.plan_placed(self.plan, ids, self.placement)
+                status, _ = zb.plan_status(self.plan)
+                self.w_ref, replaced = w, changes > 0
+            elif forced or decide(self.strategy, True, drift, self.delta):
                 zb.plan(self.plan, ids)
                 status, _ = zb.plan_status(self.plan)
                 replaced, changes = True, self._adopt(w)

@@ -35,7 +35,8 @@ STATS_LEN = 8
 
 EXPORTS = ("zb_strerror", "zb_validate", "zb_workspace_bytes", "zb_plan", "zb_plan_placed",
            "zb_plan_status", "zb_dispatch", "zb_combine", "zb_merge_workspace_bytes",
-           "zb_merge", "zb_dispatch_merged", "zb_combine_reduce", "zb_combine_merged")
+           "zb_merge", "zb_dispatch_merged", "zb_combine_reduce", "zb_combine_merged",
+           "zb_recalibrate_workspace_bytes", "zb_recalibrate")
 
 
 class ZbError(RuntimeError):
@@ -91,6 +92,11 @@ def load() -> ctypes.CDLL:
         lib.zb_dispatch_merged.argtypes = [cfgp, planp, mergep, vp, vp, vp]
         lib.zb_combine_reduce.argtypes = [cfgp, planp, mergep, vp, vp, vp, vp]
         lib.zb_combine_merged.argtypes = [cfgp, planp, mergep, vp, vp, vp]
+        lib.zb_recalibrate_workspace_bytes.argtypes = [cfgp, ctypes.c_int]
+        lib.zb_recalibrate_workspace_bytes.restype = ctypes.c_size_t
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        lib.zb_recalibrate.argtypes = [cfgp, vp, vp, ctypes.c_int, ctypes.c_float, ctypes.c_int,
+                                       vp, ctypes.c_size_t, vp, i32p, i32p]
         _lib = lib
     return _lib
 
@@ -310,3 +316,30 @@ def combine_merged(p: Plan, m: Merge, part: torch.Tensor, out: torch.Tensor,
                                   part.data_ptr(), out.data_ptr(), _stream(stream))
     if st != OK:
         raise ZbError(st, "zb_combine_merged")
+
+
+RECAL_SLOT = 0   # ViBE incremental update: one helper slot takes another expert
+RECAL_INTRA = 1  # Zepp eq. (4): two slots of one node exchange their experts
+
+
+def recalibrate(cfg: Config, cnt: torch.Tensor, placement: torch.Tensor, mode: int = RECAL_SLOT,
+                eps: float = 0.03, max_swaps: int = 64, stream=None) -> tuple[int, int]:
+    """Placement recalibration between invocations (synchronises the stream).
+    ``cnt`` int32 [P,E] (route counts, e.g. a plan's ``cnt``), ``placement``
+    int32 [P,R], changed in place.  Returns (steps taken, final max load)."""
+    _check(cnt, (cfg.P, cfg.E), torch.int32, "cnt")
+    _check(placement, (cfg.P, cfg.R), torch.int32, "placement")
+    lib = load()
+    nbytes = int(lib.zb_recalibrate_workspace_bytes(ctypes.byref(cfg.c()), int(mode)))
+    if nbytes == 0:
+        raise ZbError(ERR_INVALID, "zb_recalibrate_workspace_bytes")
+    ws = torch.empty((nbytes + 256,), dtype=torch.uint8, device=cnt.device)
+    ws_ptr = (ws.data_ptr() + 255) & ~255
+    swaps, mx = ctypes.c_int32(0), ctypes.c_int32(0)
+    st = lib.zb_recalibrate(ctypes.byref(cfg.c()), cnt.data_ptr(),
+                            placement.data_ptr() if placement.numel() else None, int(mode),
+                            float(eps), int(max_swaps), ws_ptr, nbytes, _stream(stream),
+                            ctypes.byref(swaps), ctypes.byref(mx))
+    if st != OK:
+        raise ZbError(st, "zb_recalibrate")
+    return int(swaps.value), int(mx.value)
