@@ -85,6 +85,8 @@ def _load():
         lib.zbo_merge.restype = None
         lib.zbo_dispatch_merged.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp]
         lib.zbo_dispatch_merged.restype = None
+        lib.zbo_place_by_demand.argtypes = [ctypes.POINTER(_Cfg), vp, _P32, _P32]
+        lib.zbo_place_by_demand.restype = ctypes.c_int
         lib.zbo_recalibrate.argtypes = [ctypes.POINTER(_Cfg), _P32, _P32, ctypes.c_int,
                                         ctypes.c_double, ctypes.c_int, _P32]
         lib.zbo_recalibrate.restype = ctypes.c_int
@@ -231,6 +233,19 @@ def dispatch_merged(cfg: Config, tok_row: np.ndarray, hidden_bits: np.ndarray,
     _load().zbo_dispatch_merged(ctypes.byref(cfg.c()), tok_row.ctypes.data,
                                 hidden_bits.ctypes.data, tbuf_bits.ctypes.data)
     return tbuf_bits
+
+
+def place_by_demand(cfg: Config, demand: np.ndarray, with_blocked: bool = False):
+    """Replica placement [P,R] from historical per-expert demand (int64 [E]);
+    with ``with_blocked`` also the number of picks that fit nowhere."""
+    demand = np.ascontiguousarray(demand, dtype=np.int64)
+    pl = np.zeros((cfg.P, cfg.R), np.int32)
+    blocked = np.zeros(1, np.int32)
+    st = _load().zbo_place_by_demand(ctypes.byref(cfg.c()), demand.ctypes.data, _ptr(pl),
+                                     _ptr(blocked))
+    if st != OK:
+        raise ValueError(f"zbo_place_by_demand: status {st}")
+    return (pl, int(blocked[0])) if with_blocked else pl
 
 
 def recalibrate(cfg: Config, cnt: np.ndarray, placement: np.ndarray, mode: int, eps: float,

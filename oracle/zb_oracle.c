@@ -643,6 +643,92 @@ int zbo_plan_placed(const zbo_config *c, const int32_t *ids, const int32_t *plac
   return status;
 }
 
+/* -------------------------------------- placement from historical demand */
+
+/* Whether rank r holds a copy of expert e (home or a helper slot). */
+static int rank_holds(const zbo_config *c, const int32_t *pl, int r, int e) {
+  if (home_of(c, e) == r) return 1;
+  for (int s = 0; s < c->R; s++)
+    if (pl[r * c->R + s] == e) return 1;
+  return 0;
+}
+
+/* A rank of node nd, from GPU index g0 on, with a free slot and no copy of e;
+ * -1 if none. */
+static int node_rank_for(const zbo_config *c, const int32_t *pl, int nd, int g0, int e) {
+  const int g = c->gpus_per_node;
+  for (int t = 0; t < g; t++) {
+    int r = nd * g + (g0 + t) % g;
+    if (rank_holds(c, pl, r, e)) continue;
+    for (int s = 0; s < c->R; s++)
+      if (pl[r * c->R + s] < 0) return r;
+  }
+  return -1;
+}
+
+/* Replica placement from historical demand [ZEPP 4.1: R extra slots per GPU
+ * go greedily to the experts with the highest historical token demand per
+ * replica; replicas are spread round-robin across nodes first, then within a
+ * node across GPUs, for node-level coverage].  demand[e] >= 0 (e.g. rows
+ * routed to e over past invocations).  Each of up to P*R picks takes the
+ * expert with the largest demand per copy D_e / n_e (n_e copies so far, the
+ * home copy included; compared exactly as D_a * n_b > D_b * n_a; ties to the
+ * lowest e) among experts that still fit somewhere.  The copy goes to the
+ * first node from a round-robin cursor that holds no copy of e and has a rank
+ * that can take it, else the first node from the cursor with such a rank;
+ * within the node, the first such rank from the node's own cursor; the lowest
+ * free slot.  Both cursors then move past the choice.  An expert that fits
+ * nowhere is skipped from then on (counted in *blocked); slots no expert fits
+ * stay empty.  Returns ZBO_OK or ZBO_ERR_INVALID. */
+int zbo_place_by_demand(const zbo_config *c, const int64_t *demand, int32_t *placement,
+                        int32_t *blocked) {
+  if (zbo_validate(c)) return ZBO_ERR_INVALID;
+  const int P = c->P, E = c->E, R = c->R, g = c->gpus_per_node, nodes = P / g;
+  for (int e = 0; e < E; e++)
+    if (demand[e] < 0) return ZBO_ERR_INVALID;
+  for (int x = 0; x < P * R; x++) placement[x] = -1;
+  if (blocked) *blocked = 0;
+  int64_t *n = malloc(sizeof(int64_t) * (size_t)E);
+  int *full = calloc((size_t)E, sizeof(int));
+  int *gcur = calloc((size_t)nodes, sizeof(int));
+  for (int e = 0; e < E; e++) n[e] = 1;
+  int ncur = 0;
+  for (int placed = 0; placed < P * R;) {
+    int pick = -1;
+    for (int e = 0; e < E; e++) {
+      if (full[e]) continue;
+      if (pick < 0 || demand[e] * n[pick] > demand[pick] * n[e]) pick = e;
+    }
+    if (pick < 0) break;
+    int nd = -1, r = -1;
+    for (int pass = 0; pass < 2 && r < 0; pass++)
+      for (int t = 0; t < nodes && r < 0; t++) {
+        int cand = (ncur + t) % nodes;
+        if (pass == 0) {
+          int covered = 0;
+          for (int q = cand * g; q < (cand + 1) * g; q++) covered |= rank_holds(c, placement, q, pick);
+          if (covered) continue;
+        }
+        int rr = node_rank_for(c, placement, cand, gcur[cand], pick);
+        if (rr >= 0) { nd = cand; r = rr; }
+      }
+    if (r < 0) {
+      full[pick] = 1;
+      if (blocked) *blocked += 1;
+      continue;
+    }
+    int s = 0;
+    while (placement[r * R + s] >= 0) s++;
+    placement[r * R + s] = pick;
+    n[pick] += 1;
+    ncur = (nd + 1) % nodes;
+    gcur[nd] = (r - nd * g + 1) % g;
+    placed++;
+  }
+  free(n); free(full); free(gcur);
+  return ZBO_OK;
+}
+
 /* ------------------------------------------ placement recalibration */
 
 /* Max rank load of the kept-placement plan (greedy_placed over `placement`)
