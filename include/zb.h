@@ -344,6 +344,23 @@ ZB_API int zb_combine_reduce(const zb_config *cfg, const zb_plan_t *plan, const 
 ZB_API int zb_combine_merged(const zb_config *cfg, const zb_plan_t *plan, const zb_merge_t *merge,
                              const uint16_t *part, uint16_t *out, void *stream);
 
+/* A replica placement from historical demand (Zepp, 4.1 Expert Placement and
+ * Token Routing: the R slots of each GPU go greedily to the experts with the
+ * highest historical demand per replica, spread round-robin across nodes
+ * first, then across a node's GPUs, for node-level coverage).  HOST memory:
+ * demand int64 [E] >= 0 (e.g. rows routed to each expert over past
+ * invocations), placement int32 [P][R] (written; -1 = empty), for use with
+ * zb_plan_placed.  Each pick takes the expert with the largest demand per copy
+ * D_e / n_e (n_e its copies so far, home included; exact comparison; ties to
+ * the lowest id) among experts that still fit.  The copy goes to the first
+ * node, from a round-robin cursor, that holds no copy of the expert and has a
+ * GPU that can take it, else to the first node from the cursor with such a
+ * GPU; within the node, the first such GPU from the node's own cursor; the
+ * lowest free slot.  Both cursors then move past the choice.  An expert that
+ * fits nowhere is not picked again; slots nothing fits stay empty.  Touches no
+ * device.  ZB_OK, or ZB_ERR_INVALID for a bad argument or negative demand. */
+ZB_API int zb_place_by_demand(const zb_config *cfg, const int64_t *demand, int32_t *placement);
+
 /* Placement recalibration between invocations (not part of an invocation's
  * path).  From the replica placement `placement` (device int32 [P][R], -1 =
  * empty; changed in place) and the route counts `cnt` (device int32 [P][E],

@@ -42,6 +42,7 @@ def test_replanner_plans_match_oracle(cuda_device, strategy):
     rp = replan.Replanner(zc, cuda_device, strategy, delta=0.01)
     placement = None
     replaced_later = 0
+    hist = []
     for t in range(12):
         ids, _ = synth.routing(wl, 0, t)
         w_ref_before = rp.w_ref
@@ -49,7 +50,16 @@ def test_replanner_plans_match_oracle(cuda_device, strategy):
         w = np.bincount(ids.ravel(), minlength=wl.E)
         if rep.drift is not None:
             assert rep.drift == pytest.approx(replan.cosine_drift(w, w_ref_before), abs=1e-12)
-        if strategy == "incremental" and t > 0:
+        if strategy == "history":
+            # placed from the summed counts of the last 10 invocations, at
+            # t = 0 (its own counts) and t = 10
+            if t % 10 == 0:
+                past = hist[-10:] if t else [w]
+                placement = oracle.place_by_demand(oc, np.sum(past, axis=0).astype(np.int64))
+            o = oracle.plan(oc, ids, want_M=False, placement=placement)
+            hist.append(w)
+            replaced_later += rep.replaced and t > 0
+        elif strategy == "incremental" and t > 0:
             # recalibrated from the kept placement when drift or capacity asks
             kept = oracle.plan(oc, ids, want_M=False, placement=placement)
             if rep.drift > 0.01 or kept["status"] == oracle.ERR_CAPACITY:
@@ -71,5 +81,7 @@ def test_replanner_plans_match_oracle(cuda_device, strategy):
         assert replaced_later == 11
     elif strategy == "incremental":
         assert replaced_later > 0
+    elif strategy == "history":
+        assert replaced_later == 1
     else:
         assert 0 < replaced_later < 11

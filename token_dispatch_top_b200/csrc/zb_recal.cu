@@ -1,12 +1,20 @@
-// zb_recal.cu -- zb_recalibrate: placement recalibration between invocations.
-// The only call besides zb_plan_status that synchronises its stream: every
-// step reads the scores of all candidates back to the host to pick one, and
-// the host keeps the placement being changed (in host memory it allocates).
+// zb_recal.cu -- replica placement between invocations.
+//   zb_place_by_demand  a placement from historical per-expert demand (host
+//                       only: a few hundred picks over at most 384 experts)
+//   zb_recalibrate      recalibration of a kept placement; with
+//                       zb_plan_status the only calls that synchronise their
+//                       stream: every step reads the scores of all candidates
+//                       back to the host to pick one, and the host keeps the
+//                       placement being changed (in host memory it allocates)
 //
-// Sources: ViBE, "Drift-Aware Recalibration" (incremental placement update:
+// Sources: Zepp, "4.1 Expert Placement and Token Routing" (R slots per GPU
+// given to the experts of highest historical demand per replica, spread
+// round-robin over nodes, then over a node's GPUs); ViBE, "Drift-Aware
+// Recalibration" (incremental placement update:
 // from the current placement, minimal cross-GPU expert swaps until every GPU
 // is within eps of the mean); Zepp, "4.3 Three-Stream Scheduling", eq. (4)
 // (intra-node swaps of expert replicas that keep node-level coverage).
+#include <algorithm>
 #include <climits>
 #include <cstring>
 #include <vector>
@@ -52,9 +60,116 @@ RecalLayout recal_layout(const zb_config& c, int mode) {
   return w;
 }
 
+// Demand-per-copy placement state: copies so far per expert, and the
+// round-robin cursors over nodes and over each node's GPUs.
+class DemandPlacer {
+ public:
+  DemandPlacer(const zb_config& c, const int64_t* demand, int32_t* pl)
+      : c_(c), d_(demand), pl_(pl), copies_(size_t(c.E), 1), skip_(size_t(c.E), false),
+        gcur_(size_t(c.P / c.gpus_per_node), 0) {}
+
+  void run() {
+    const int slots = c_.P * c_.R;
+    std::fill(pl_, pl_ + slots, -1);
+    int filled = 0;
+    while (filled < slots) {
+      const int e = most_deserving();
+      if (e < 0) return;  // no expert fits anywhere: the rest stays empty
+      if (place(e))
+        ++filled;
+      else
+        skip_[size_t(e)] = true;
+    }
+  }
+
+ private:
+  // The expert with the largest demand per copy D_e / n_e (exact: compare
+  // D_a * n_b with D_b * n_a), the lowest id among equals.
+  int most_deserving() const {
+    int best = -1;
+    for (int e = 0; e < c_.E; ++e) {
+      if (skip_[size_t(e)]) continue;
+      if (best < 0 || d_[e] * copies_[size_t(best)] > d_[best] * copies_[size_t(e)]) best = e;
+    }
+    return best;
+  }
+
+  bool holds(int r, int e) const {
+    if (e / (c_.E / c_.P) == r) return true;
+    for (int s = 0; s < c_.R; ++s)
+      if (pl_[r * c_.R + s] == e) return true;
+    return false;
+  }
+
+  bool has_free_slot(int r) const {
+    for (int s = 0; s < c_.R; ++s)
+      if (pl_[r * c_.R + s] < 0) return true;
+    return false;
+  }
+
+  // First GPU of node nd, from that node's cursor, that can take e.
+  int rank_in_node(int nd, int e) const {
+    const int g = c_.gpus_per_node;
+    for (int t = 0; t < g; ++t) {
+      const int r = nd * g + (gcur_[size_t(nd)] + t) % g;
+      if (!holds(r, e) && has_free_slot(r)) return r;
+    }
+    return -1;
+  }
+
+  bool node_covers(int nd, int e) const {
+    const int g = c_.gpus_per_node;
+    for (int r = nd * g; r < nd * g + g; ++r)
+      if (holds(r, e)) return true;
+    return false;
+  }
+
+  // Nodes from the cursor: one without a copy of e first, then any; within
+  // the node, its GPUs from its own cursor; the lowest free slot.
+  bool place(int e) {
+    const int g = c_.gpus_per_node, nodes = c_.P / g;
+    int nd = -1, r = -1;
+    for (int pass = 0; pass < 2 && r < 0; ++pass)
+      for (int t = 0; t < nodes && r < 0; ++t) {
+        const int cand = (ncur_ + t) % nodes;
+        if (pass == 0 && node_covers(cand, e)) continue;
+        const int rr = rank_in_node(cand, e);
+        if (rr >= 0) {
+          nd = cand;
+          r = rr;
+        }
+      }
+    if (r < 0) return false;
+    int s = 0;
+    while (pl_[r * c_.R + s] >= 0) ++s;
+    pl_[r * c_.R + s] = e;
+    ++copies_[size_t(e)];
+    ncur_ = (nd + 1) % nodes;
+    gcur_[size_t(nd)] = (r - nd * g + 1) % g;
+    return true;
+  }
+
+  const zb_config& c_;
+  const int64_t* d_;
+  int32_t* pl_;
+  std::vector<int64_t> copies_;
+  std::vector<bool> skip_;
+  std::vector<int> gcur_;
+  int ncur_ = 0;
+};
+
 }  // namespace
 
 extern "C" {
+
+int zb_place_by_demand(const zb_config* c, const int64_t* demand, int32_t* placement) {
+  if (zb_validate(c) != ZB_OK || !demand || (c->R > 0 && !placement)) return ZB_ERR_INVALID;
+  for (int e = 0; e < c->E; ++e)
+    if (demand[e] < 0) return ZB_ERR_INVALID;
+  if (c->R == 0) return ZB_OK;
+  DemandPlacer(*c, demand, placement).run();
+  return ZB_OK;
+}
 
 size_t zb_recalibrate_workspace_bytes(const zb_config* c, int mode) {
   if (zb_validate(c) != ZB_OK || (mode != 0 && mode != 1)) return 0;

@@ -16,7 +16,11 @@ pages weigh this three ways:
   this invocation's per-expert load w and the load the placement was made for
   exceeds delta (ViBE, drift detection, delta = 0.05), or when the kept
   placement no longer fits the receive buffers;
-* ``incremental`` - the same trigger, but instead of a fresh placement the
+* ``history`` - Zepp's history-based placement (4.1): the slots go to the
+  experts with the highest demand per replica over the last ``window``
+  invocations (zb_place_by_demand), placed first at invocation 0 and again
+  every ``window`` invocations; quotas are re-split on every invocation;
+* ``incremental`` - the drift trigger, but instead of a fresh placement the
   kept one is recalibrated (ViBE's incremental update, zb_recalibrate mode
   0): one helper slot changes per step until every rank is within eps = 0.03
   of the mean or no change helps, so only the changed slots move weights.
@@ -38,7 +42,7 @@ import torch
 
 from . import zb
 
-STRATEGIES = ("every", "static", "drift", "incremental")
+STRATEGIES = ("every", "static", "drift", "incremental", "history")
 
 
 def cosine_drift(w: np.ndarray, w_ref: np.ndarray) -> float:
@@ -66,7 +70,7 @@ def decide(strategy: str, have_placement: bool, drift: float | None, delta: floa
         raise ValueError(f"unknown strategy {strategy!r}")
     if not have_placement or strategy == "every":
         return True
-    if strategy == "static":
+    if strategy in ("static", "history"):
         return False
     return drift is not None and drift > delta  # drift and incremental
 
@@ -85,11 +89,13 @@ class Replanner:
     """Plans a stream of invocations of one shape under a placement policy."""
 
     def __init__(self, cfg: zb.Config, device, strategy: str = "drift", delta: float = 0.05,
-                 eps: float = 0.03, max_swaps: int = 64):
+                 eps: float = 0.03, max_swaps: int = 64, window: int = 10):
         if strategy not in STRATEGIES:
             raise ValueError(f"unknown strategy {strategy!r}")
         self.cfg, self.strategy, self.delta = cfg, strategy, delta
-        self.eps, self.max_swaps = eps, max_swaps
+        self.eps, self.max_swaps, self.window = eps, max_swaps, window
+        self.history: list[np.ndarray] = []  # per-expert loads of recent invocations
+        self.count = 0
         self.plan = zb.Plan(cfg, device, with_row_src=False)
         self.placement: torch.Tensor | None = None
         self.w_ref: np.ndarray | None = None
@@ -101,7 +107,34 @@ class Replanner:
         self.placement, self.w_ref = new, w
         return changes
 
+    def _history_step(self, ids: torch.Tensor) -> StepReport:
+        """Zepp: place from the demand of the last `window` invocations."""
+        replaced, changes = False, 0
+        if self.placement is None:
+            # the first invocation has no history: its own counts stand in
+            zb.plan(self.plan, ids)
+            zb.plan_status(self.plan)
+            self.history.append(self.plan.cnt.sum(0).cpu().numpy())
+        if self.count % self.window == 0:
+            demand = np.sum(self.history[-self.window:], axis=0).astype(np.int64)
+            new = torch.from_numpy(zb.place_by_demand(self.cfg, demand)).to(self.plan.cnt.device)
+            changes = slot_changes(None if self.placement is None else
+                                   self.placement.cpu().numpy(), new.cpu().numpy())
+            self.placement, replaced = new, True
+        zb.plan_placed(self.plan, ids, self.placement)
+        status, _ = zb.plan_status(self.plan)
+        if self.count > 0:
+            self.history.append(self.plan.cnt.sum(0).cpu().numpy())
+        self.history = self.history[-self.window:]
+        self.count += 1
+        st = self.plan.stats.cpu().numpy()
+        return StepReport(status=int(status), max_load=int(st[zb.STAT_MAX_LOAD]),
+                          water_level=int(st[zb.STAT_WATER_LEVEL]), replaced=replaced,
+                          slot_changes=changes, drift=None)
+
     def step(self, ids: torch.Tensor) -> StepReport:
+        if self.strategy == "history":
+            return self._history_step(ids)
         drift = None
         if self.placement is None or self.strategy == "every":
             zb.plan(self.plan, ids)

@@ -13,6 +13,7 @@ import math
 import os
 from dataclasses import dataclass
 
+import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -36,7 +37,7 @@ STATS_LEN = 8
 EXPORTS = ("zb_strerror", "zb_validate", "zb_workspace_bytes", "zb_plan", "zb_plan_placed",
            "zb_plan_status", "zb_dispatch", "zb_combine", "zb_merge_workspace_bytes",
            "zb_merge", "zb_dispatch_merged", "zb_combine_reduce", "zb_combine_merged",
-           "zb_recalibrate_workspace_bytes", "zb_recalibrate")
+           "zb_recalibrate_workspace_bytes", "zb_recalibrate", "zb_place_by_demand")
 
 
 class ZbError(RuntimeError):
@@ -97,6 +98,7 @@ def load() -> ctypes.CDLL:
         i32p = ctypes.POINTER(ctypes.c_int32)
         lib.zb_recalibrate.argtypes = [cfgp, vp, vp, ctypes.c_int, ctypes.c_float, ctypes.c_int,
                                        vp, ctypes.c_size_t, vp, i32p, i32p]
+        lib.zb_place_by_demand.argtypes = [cfgp, vp, vp]
         _lib = lib
     return _lib
 
@@ -343,3 +345,17 @@ def recalibrate(cfg: Config, cnt: torch.Tensor, placement: torch.Tensor, mode: i
     if st != OK:
         raise ZbError(st, "zb_recalibrate")
     return int(swaps.value), int(mx.value)
+
+
+def place_by_demand(cfg: Config, demand) -> np.ndarray:
+    """Replica placement int32 [P,R] from historical per-expert demand (host
+    int64 [E]); runs on the host, for zb.plan_placed."""
+    d = np.ascontiguousarray(np.asarray(demand), dtype=np.int64)
+    if d.shape != (cfg.E,):
+        raise ValueError(f"demand: expected shape ({cfg.E},), got {d.shape}")
+    pl = np.full((cfg.P, cfg.R), -1, np.int32)
+    st = load().zb_place_by_demand(ctypes.byref(cfg.c()), d.ctypes.data,
+                                   pl.ctypes.data if pl.size else None)
+    if st != OK:
+        raise ZbError(st, "zb_place_by_demand")
+    return pl
