@@ -121,7 +121,7 @@ template <int K>
 cudaError_t combine_k(int ntok, int H, int64_t nrows, const int32_t* dst_row,
                       const int64_t* stats, const uint16_t* y, const float* w, uint16_t* out,
                       cudaStream_t s) {
-  constexpr int U = K <= 6 ? 4 : (K <= 8 ? 2 : 1);
+  constexpr int U = K <= 6 ? 4 : (K <= 16 ? 2 : 1);
   const int blocks = (ntok + kMoveWarps - 1) / kMoveWarps;
   k_combine<K, U><<<blocks, kMoveThreads, 0, s>>>(ntok, H, nrows, dst_row, stats,
                                                   reinterpret_cast<const uint4*>(y), w,
