@@ -299,6 +299,20 @@ def test_maximum_shape(dev):
     _run_small(dev, ids, E=E, R=2, H=64, gpn=1, cap_rows=S * K * P)
 
 
+@pytest.mark.parametrize("K", [7, 9, 12, 13, 14, 16])
+def test_large_k_two_vectors_in_flight(dev, K):
+    """K = 7..16 combine with two vectors per row in flight: H = 1032 is 129
+    vectors, so each lane runs both vectors and the last chunk is ragged."""
+    rng = np.random.default_rng(40 + K)
+    P, E, S, H = 4, 32, 70, 1032
+    ids = rng.integers(0, E, (P, S, K)).astype(np.int32)
+    kw = dict(P=P, E=E, K=K, S=S, H=H, R=2, cap_rows=P * S * K)
+    zc, oc = zb.Config(**kw), oracle.Config(**kw)
+    w = rng.dirichlet(np.ones(K), size=(P, S)).astype(np.float32)
+    full_parity(zc, oc, ids, w, _rand_bits(rng, (P, S, H)), _rand_bits(rng, (P * zc.cap, H)),
+                dev, with_row_src=False)
+
+
 def test_all_rows_on_one_expert_and_duplicates(dev):
     _run_small(dev, np.zeros((8, 64, 4), np.int32), E=16, R=7)
     rng = np.random.default_rng(5)
