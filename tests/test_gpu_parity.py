@@ -299,18 +299,44 @@ def test_maximum_shape(dev):
     _run_small(dev, ids, E=E, R=2, H=64, gpn=1, cap_rows=S * K * P)
 
 
-@pytest.mark.parametrize("K", [7, 9, 12, 13, 14, 16])
-def test_large_k_two_vectors_in_flight(dev, K):
-    """K = 7..16 combine with two vectors per row in flight: H = 1032 is 129
-    vectors, so each lane runs both vectors and the last chunk is ragged."""
+@pytest.mark.parametrize("K,H", [(7, 1032), (9, 1032), (12, 1032), (13, 1032), (14, 1032),
+                                 (16, 1032), (7, 1040), (8, 1040), (12, 1040), (16, 1040)])
+def test_large_k_two_vectors_in_flight(dev, K, H):
+    """K = 7..16 combine.  H = 1032 (not a multiple of 16): 16-byte vectors,
+    two per row in flight, 129 per row with a ragged last chunk.  H = 1040:
+    the 32-byte kernel, 65 vectors per row, also ragged."""
     rng = np.random.default_rng(40 + K)
-    P, E, S, H = 4, 32, 70, 1032
+    P, E, S = 4, 32, 70
     ids = rng.integers(0, E, (P, S, K)).astype(np.int32)
     kw = dict(P=P, E=E, K=K, S=S, H=H, R=2, cap_rows=P * S * K)
     zc, oc = zb.Config(**kw), oracle.Config(**kw)
     w = rng.dirichlet(np.ones(K), size=(P, S)).astype(np.float32)
     full_parity(zc, oc, ids, w, _rand_bits(rng, (P, S, H)), _rand_bits(rng, (P * zc.cap, H)),
                 dev, with_row_src=False)
+
+
+def test_combine_on_16_byte_aligned_buffers(dev):
+    """y and out 16- but not 32-byte aligned: K = 8 takes the 16-byte kernel,
+    bit for bit the same as the 32-byte one on aligned copies."""
+    rng = np.random.default_rng(8)
+    P, E, K, S, H = 4, 32, 8, 50, 1024
+    ids = rng.integers(0, E, (P, S, K)).astype(np.int32)
+    zc = zb.Config(P=P, E=E, K=K, S=S, H=H, R=1, cap_rows=P * S * K)
+    p, status, _ = gpu_plan(zc, ids, dev, with_row_src=False)
+    assert status >= 0
+    w = torch.from_numpy(rng.dirichlet(np.ones(K), size=(P, S)).astype(np.float32)).to(dev)
+    y_a = bits_to_bf16(_rand_bits(rng, (P, zc.cap, H)), dev)
+    y_raw = torch.empty(y_a.numel() + 8, dtype=torch.bfloat16, device=dev)
+    y_u = y_raw[8:].view(P, zc.cap, H)  # 16-byte offset
+    y_u.copy_(y_a)
+    out_raw = torch.empty(P * S * H + 8, dtype=torch.bfloat16, device=dev)
+    out_u = out_raw[8:].view(P, S, H)
+    out_a = torch.empty((P, S, H), dtype=torch.bfloat16, device=dev)
+    assert y_u.data_ptr() % 32 == 16 and out_u.data_ptr() % 32 == 16
+    zb.combine(p, y_a, w, out_a)
+    zb.combine(p, y_u, w, out_u)
+    torch.cuda.synchronize()
+    assert torch.equal(out_a.view(torch.int16), out_u.view(torch.int16))
 
 
 def test_all_rows_on_one_expert_and_duplicates(dev):

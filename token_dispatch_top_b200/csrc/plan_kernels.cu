@@ -13,6 +13,8 @@
 // stages 1, 2, 3, 5); Zepp "4.1 Expert Placement and Token Routing" (R slots
 // per GPU, node-first placement, eq. (1)); MoonEP "What MoonEP enforces and
 // how" (S x K per rank, cu_seqlens, expert-grouped fixed buffers).
+#include <atomic>
+
 #include "zb_internal.cuh"
 
 namespace zb {
@@ -980,16 +982,16 @@ cudaError_t launch_hist(const PlanArgs& a, cudaStream_t s) {
 
 template <int kMode, bool kRepair, bool kBand>
 cudaError_t launch_planner_mode(const PlanArgs& a, size_t smem, cudaStream_t s) {
-  static bool configured[64] = {};
+  static std::atomic<bool> configured[64];
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
+  if (!configured[dev].load(std::memory_order_acquire)) {
     err = cudaFuncSetAttribute(k_planner<kMode, kRepair, kBand>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     if (err != cudaSuccess) return err;
-    configured[dev] = true;
+    configured[dev].store(true, std::memory_order_release);
   }
   k_planner<kMode, kRepair, kBand><<<1, kPlanThreads, smem, s>>>(a);
   return cudaGetLastError();
@@ -1018,16 +1020,16 @@ size_t eval_smem_bytes(int P, int E, int R) {
 cudaError_t launch_eval_placements(const EvalArgs& ea, cudaStream_t s) {
   if (ea.ncand == 0) return cudaSuccess;
   const size_t smem = eval_smem_bytes(ea.P, ea.E, ea.R);
-  static bool configured[64] = {};
+  static std::atomic<bool> configured[64];
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
+  if (!configured[dev].load(std::memory_order_acquire)) {
     err = cudaFuncSetAttribute(k_eval_placements, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                200 * 1024);
     if (err != cudaSuccess) return err;
-    configured[dev] = true;
+    configured[dev].store(true, std::memory_order_release);
   }
   const int64_t blocks = (ea.ncand + kEvalWarps - 1) / kEvalWarps;
   k_eval_placements<<<unsigned(blocks), kEvalThreads, smem, s>>>(ea);

@@ -13,6 +13,25 @@ namespace zb {
 __device__ __forceinline__ uint4 ld_nc(const uint4* p) { return __ldcs(p); }
 __device__ __forceinline__ void st_v4(uint4* p, const uint4& v) { __stcs(p, v); }
 
+// 32-byte vectors (sm_100's 256-bit global accesses): 16 bf16 per lane.
+struct alignas(32) V8 {
+  uint32_t v[8];
+};
+__device__ __forceinline__ V8 ld_nc8(const V8* p) {
+  V8 r;
+  asm volatile("ld.global.cs.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r.v[0]), "=r"(r.v[1]), "=r"(r.v[2]), "=r"(r.v[3]), "=r"(r.v[4]),
+                 "=r"(r.v[5]), "=r"(r.v[6]), "=r"(r.v[7])
+               : "l"(p));
+  return r;
+}
+__device__ __forceinline__ void st_v8(V8* p, const V8& r) {
+  asm volatile("st.global.cs.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(r.v[0]),
+               "r"(r.v[1]), "r"(r.v[2]), "r"(r.v[3]), "r"(r.v[4]), "r"(r.v[5]), "r"(r.v[6]),
+               "r"(r.v[7])
+               : "memory");
+}
+
 // bf16 widens to float exactly: it is the upper half of a binary32.
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
