@@ -300,11 +300,11 @@ def test_maximum_shape(dev):
 
 
 @pytest.mark.parametrize("K,H", [(7, 1032), (9, 1032), (12, 1032), (13, 1032), (14, 1032),
-                                 (16, 1032), (7, 1040), (8, 1040), (12, 1040), (16, 1040)])
+                                 (16, 1032), (8, 1040), (16, 1040), (7, 4112), (8, 4112)])
 def test_large_k_two_vectors_in_flight(dev, K, H):
-    """K = 7..16 combine.  H = 1032 (not a multiple of 16): 16-byte vectors,
-    two per row in flight, 129 per row with a ragged last chunk.  H = 1040:
-    the 32-byte kernel, 65 vectors per row, also ragged."""
+    """K = 7..16 combine.  H = 1032 and 1040: 16-byte vectors, two per row in
+    flight, with a ragged last chunk.  H = 4112 at K = 7 and 8: the 32-byte
+    kernel, 257 vectors per row, also ragged."""
     rng = np.random.default_rng(40 + K)
     P, E, S = 4, 32, 70
     ids = rng.integers(0, E, (P, S, K)).astype(np.int32)
@@ -319,7 +319,7 @@ def test_combine_on_16_byte_aligned_buffers(dev):
     """y and out 16- but not 32-byte aligned: K = 8 takes the 16-byte kernel,
     bit for bit the same as the 32-byte one on aligned copies."""
     rng = np.random.default_rng(8)
-    P, E, K, S, H = 4, 32, 8, 50, 1024
+    P, E, K, S, H = 4, 32, 8, 50, 4096
     ids = rng.integers(0, E, (P, S, K)).astype(np.int32)
     zc = zb.Config(P=P, E=E, K=K, S=S, H=H, R=1, cap_rows=P * S * K)
     p, status, _ = gpu_plan(zc, ids, dev, with_row_src=False)

@@ -4,8 +4,8 @@
 // flight per lane, and K specialised at compile time so the K destination (or
 // source) rows are all addressed before the first access.
 //
-// The combine for K >= 7 loads 32-byte vectors when the row width and the
-// buffers allow (k_combine_wide).
+// The combine for K = 7 and 8 on wide rows (H >= 4096) loads 32-byte vectors
+// when the buffers are 32-byte aligned (k_combine_wide).
 //
 // Sources: MoonEP "What MoonEP enforces and how" (zero-copy writes into
 // fixed-shape expert-grouped buffers); Zepp "4.2 Split and Merge" (combine);
@@ -109,8 +109,9 @@ __global__ void __launch_bounds__(kMoveThreads) k_combine(int ntok, int H, int64
   }
 }
 
-// k_combine with 32-byte vectors, for K >= 7 (H % 16 == 0, y and out 32-byte
-// aligned): the same fold, half as many load instructions per row.
+// k_combine with 32-byte vectors, for K = 7 and 8 on rows of H >= 4096 (H % 16
+// == 0, y and out 32-byte aligned): the same fold, half as many load
+// instructions per row.
 template <int K>
 __global__ void __launch_bounds__(kMoveThreads) k_combine_wide(int ntok, int H, int64_t nrows,
                                                                const int32_t* __restrict__ dst_row,
@@ -174,8 +175,11 @@ cudaError_t combine_k(int ntok, int H, int64_t nrows, const int32_t* dst_row,
                       cudaStream_t s) {
   constexpr int U = K <= 6 ? 4 : (K <= 16 ? 2 : 1);
   const int blocks = (ntok + kMoveWarps - 1) / kMoveWarps;
-  if constexpr (K >= 7) {  // measured: +4% at K = 8, H = 7168; slower at K = 6
-    const bool wide_ok = (H % 16) == 0 && (reinterpret_cast<uintptr_t>(y) & 31u) == 0 &&
+  // Measured: at K = 8 the 32-byte kernel is 4% faster for H = 7168 and 3%
+  // slower for H = 2048; at K = 6, and at K >= 12 for H = 2048, it is slower.
+  if constexpr (K == 7 || K == 8) {
+    const bool wide_ok = H >= 4096 && (H % 16) == 0 &&
+                         (reinterpret_cast<uintptr_t>(y) & 31u) == 0 &&
                          (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
     if (wide_ok) {
       k_combine_wide<K><<<blocks, kMoveThreads, 0, s>>>(ntok, H, nrows, dst_row, stats,
