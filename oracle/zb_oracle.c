@@ -10,14 +10,20 @@
  *
  * Sources (web pages; each function cites the passage it follows):
  *  [ZEPP]  Zepp summary page, "Methodology / 4.1 Expert Placement and Token
- *          Routing" (R replica slots per GPU, hierarchical round-robin
- *          placement, locality-preferred routing eq. (1)).
+ *          Routing" (R replica slots per GPU given by historical demand per
+ *          replica, hierarchical round-robin placement, locality-preferred
+ *          routing eq. (1) with its relaxation C), "4.2 Split and Merge" (merge
+ *          for dispatch and combine), "4.3 Three-Stream Scheduling" (eq. (4),
+ *          intra-node swaps).
  *  [ISER]  "ISER-MoE: Dynamic In-Switch Replication of Hot Experts for Load
  *          Balancing in Expert-Parallel", "Methodology / HALO-Q Scheduler"
- *          (Objective 1 water level T, stage 1 count exchange, stage 2 greedy
- *          placement of the busiest rank's heaviest home expert, stage 3 slot
- *          colouring by the smallest free index, stage 5 local-first route
- *          rewrite), "Background" (rank imbalance R = max/mean).
+ *          (Objective 1 water level T, Objective 2 locality, stage 1 count
+ *          exchange, stage 2 greedy placement of the busiest rank's heaviest
+ *          home expert, stage 3 slot colouring by the smallest free index,
+ *          stage 4 quota repair, stage 5 local-first route rewrite),
+ *          "Background" (rank imbalance R = max/mean).
+ *  [ViBE]  ViBE, "Drift-Aware Recalibration" (incremental placement update
+ *          within a tolerance eps of the mean).
  *  [MOON]  "MoonEP: Planner-Enforced SxK Token Balance and Zero-Copy Buffers
  *          to Fix MoE Skew", "What MoonEP enforces and how" (every rank gets
  *          exactly S*K rows; the planner emits cu_seqlens; fixed-shape
