@@ -1,18 +1,26 @@
 // plan_kernels.cu -- steps 1-3 of an invocation on one GPU:
 //   k_hist     per-(source rank, chunk) expert histogram in shared memory
 //   k_planner  one CTA: route counts, water level, greedy replica placement
-//              (one warp, lanes = ranks), quotas, cu_seqlens, locality-first
-//              transport and the per-(source, expert) segment table
+//              (one warp, lanes = ranks; or the quotas over a kept
+//              placement), optional quota repair between rank pairs, quotas,
+//              cu_seqlens, locality-first transport (exact quotas or eq. (1)'s
+//              band) and the per-(source, expert) segment table; one instance
+//              per greedy mode x repair x band
 //   k_assign   per-(source rank, chunk): stable rank of every entry among the
 //              source's entries of the same expert, then its destination row
+// and, between invocations,
+//   k_eval_placements  one warp per candidate placement: the kept-placement
+//              greedy's max rank load (scores for zb_recalibrate)
 //
 // No kernel waits on another CTA: the chunk prefix each assignment CTA needs
 // is summed directly from the per-chunk histograms.
 //
-// Sources: ISER-MoE "Methodology / HALO-Q Scheduler" (Objective 1 water level,
-// stages 1, 2, 3, 5); Zepp "4.1 Expert Placement and Token Routing" (R slots
-// per GPU, node-first placement, eq. (1)); MoonEP "What MoonEP enforces and
-// how" (S x K per rank, cu_seqlens, expert-grouped fixed buffers).
+// Sources: ISER-MoE "Methodology / HALO-Q Scheduler" (Objectives 1 and 2,
+// stages 1-5); Zepp "4.1 Expert Placement and Token Routing" (R slots per GPU,
+// node-first placement, eq. (1) and its relaxation C), "4.3 Three-Stream
+// Scheduling" (eq. (4)); ViBE "Drift-Aware Recalibration"; MoonEP "What MoonEP
+// enforces and how" (S x K per rank, cu_seqlens, expert-grouped fixed
+// buffers).
 #include <atomic>
 
 #include "zb_internal.cuh"
