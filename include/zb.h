@@ -358,7 +358,8 @@ ZB_API int zb_combine_merged(const zb_config *cfg, const zb_plan_t *plan, const 
  * GPU; within the node, the first such GPU from the node's own cursor; the
  * lowest free slot.  Both cursors then move past the choice.  An expert that
  * fits nowhere is not picked again; slots nothing fits stay empty.  Touches no
- * device.  ZB_OK, or ZB_ERR_INVALID for a bad argument or negative demand. */
+ * device.  ZB_OK, or ZB_ERR_INVALID for a bad argument or a demand outside
+ * [0, 2^57] (demand times copies must fit in int64). */
 ZB_API int zb_place_by_demand(const zb_config *cfg, const int64_t *demand, int32_t *placement);
 
 /* Placement recalibration between invocations (not part of an invocation's

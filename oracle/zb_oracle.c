@@ -690,8 +690,8 @@ int zbo_place_by_demand(const zbo_config *c, const int64_t *demand, int32_t *pla
                         int32_t *blocked) {
   if (zbo_validate(c)) return ZBO_ERR_INVALID;
   const int P = c->P, E = c->E, R = c->R, g = c->gpus_per_node, nodes = P / g;
-  for (int e = 0; e < E; e++)
-    if (demand[e] < 0) return ZBO_ERR_INVALID;
+  for (int e = 0; e < E; e++) /* D * copies (copies <= 32) must fit in int64 */
+    if (demand[e] < 0 || demand[e] > ((int64_t)1 << 57)) return ZBO_ERR_INVALID;
   for (int x = 0; x < P * R; x++) placement[x] = -1;
   if (blocked) *blocked = 0;
   int64_t *n = malloc(sizeof(int64_t) * (size_t)E);

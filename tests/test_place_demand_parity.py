@@ -51,7 +51,13 @@ def test_largest_shape():
                                   oracle.place_by_demand(oracle.Config(**kw), D))
 
 
-def test_rejects_negative_demand():
+def test_rejects_negative_or_too_large_demand():
     zc = zb.Config(P=2, E=4, K=1, S=1, H=8, R=1)
-    with pytest.raises(zb.ZbError):
-        zb.place_by_demand(zc, np.array([1, -1, 0, 0]))
+    oc = oracle.Config(P=2, E=4, K=1, S=1, H=8, R=1)
+    for bad in ([1, -1, 0, 0], [0, 0, (1 << 57) + 1, 0]):
+        with pytest.raises(zb.ZbError):
+            zb.place_by_demand(zc, np.array(bad, np.int64))
+        with pytest.raises(ValueError):
+            oracle.place_by_demand(oc, np.array(bad, np.int64))
+    big = np.array([1 << 57, 1 << 56, 3, 0], np.int64)  # the largest accepted demand
+    np.testing.assert_array_equal(zb.place_by_demand(zc, big), oracle.place_by_demand(oc, big))

@@ -164,8 +164,8 @@ extern "C" {
 
 int zb_place_by_demand(const zb_config* c, const int64_t* demand, int32_t* placement) {
   if (zb_validate(c) != ZB_OK || !demand || (c->R > 0 && !placement)) return ZB_ERR_INVALID;
-  for (int e = 0; e < c->E; ++e)
-    if (demand[e] < 0) return ZB_ERR_INVALID;
+  for (int e = 0; e < c->E; ++e)  // D * copies (copies <= 32) must fit in int64
+    if (demand[e] < 0 || demand[e] > (int64_t(1) << 57)) return ZB_ERR_INVALID;
   if (c->R == 0) return ZB_OK;
   DemandPlacer(*c, demand, placement).run();
   return ZB_OK;
