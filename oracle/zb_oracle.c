@@ -675,7 +675,7 @@ static int node_rank_for(const zbo_config *c, const int32_t *pl, int nd, int g0,
 /* Replica placement from historical demand [ZEPP 4.1: R extra slots per GPU
  * go greedily to the experts with the highest historical token demand per
  * replica; replicas are spread round-robin across nodes first, then within a
- * node across GPUs, for node-level coverage].  demand[e] >= 0 (e.g. rows
+ * node across GPUs, for node-level coverage].  0 <= demand[e] <= 2^57 (e.g. rows
  * routed to e over past invocations).  Each of up to P*R picks takes the
  * expert with the largest demand per copy D_e / n_e (n_e copies so far, the
  * home copy included; compared exactly as D_a * n_b > D_b * n_a; ties to the
