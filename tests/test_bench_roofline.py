@@ -1,0 +1,52 @@
+"""bench.py's roofline inputs, on CPU.
+
+* algorithmic_bytes on the mid workload equals the per-step figures stated in
+  the design notes (940.3 MB dispatch, 941.1 MB combine) and the closed forms
+  P*S*H*2 + N*H*2 + 4N and N*H*2 + 8N + P*S*H*2, recomputed here.
+* recorded_traffic reports the committed ncu DRAM bytes only while the sources
+  they were measured on hash to the recorded value, and None for a changed
+  source, a missing file or an unknown kernel.
+* the peak comes from the measured peaks file when present.
+"""
+import json
+import os
+
+import bench
+from token_dispatch_top_b200 import synth
+
+
+def test_algorithmic_bytes_mid():
+    wl = synth.WORKLOADS["mid"]
+    P, S, K, H = wl.P, wl.S, wl.K, wl.H
+    N = P * S * K
+    ab = bench.algorithmic_bytes(wl)
+    assert ab["dispatch"] == P * S * H * 2 + N * H * 2 + 4 * N == 940_310_528
+    assert ab["combine"] == N * H * 2 + 8 * N + P * S * H * 2 == 941_096_960
+    assert ab["plan"] == 12 * N
+
+
+def test_recorded_traffic_follows_the_source_hash(tmp_path, monkeypatch):
+    rec = json.load(open(os.path.join(bench.ROOT, "profiles", "traffic.json")))
+    assert rec["source_hash"] == bench.kernel_source_hash(rec["source_files"])
+    assert bench.recorded_traffic("k_dispatch") == rec["kernels"]["k_dispatch"][
+        "dram_bytes_per_launch"]
+    assert bench.recorded_traffic("k_nothing") is None
+    # a copy of the tree whose kernel source differs: the record no longer applies
+    csrc = tmp_path / "token_dispatch_top_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for name in rec["source_files"]:
+        data = open(os.path.join(bench.ROOT, "token_dispatch_top_b200", "csrc", name)).read()
+        (csrc / name).write_text(data + "\n// changed\n")
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic("k_dispatch") is None
+    (tmp_path / "profiles" / "traffic.json").unlink()
+    assert bench.recorded_traffic("k_dispatch") is None
+
+
+def test_peak_from_measured_file(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.read_peaks() == (bench.FALLBACK_HBM_GBS, "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6508.8}))
+    assert bench.read_peaks() == (6508.8, "measured")
