@@ -27,10 +27,24 @@ def test_algorithmic_bytes_mid():
 
 def test_recorded_traffic_follows_the_source_hash(tmp_path, monkeypatch):
     rec = json.load(open(os.path.join(bench.ROOT, "profiles", "traffic.json")))
-    assert rec["source_hash"] == bench.kernel_source_hash(rec["source_files"])
+    current = rec["source_hash"] == bench.kernel_source_hash(rec["source_files"])
+    want = rec["kernels"]["k_dispatch"]["dram_bytes_per_launch"] if current else None
+    assert bench.recorded_traffic("k_dispatch") == want
+    assert bench.recorded_traffic("k_nothing") is None
+    # a copy of the tree with the recorded sources: the record applies
+    same = tmp_path / "same"
+    (same / "token_dispatch_top_b200" / "csrc").mkdir(parents=True)
+    for name in rec["source_files"]:
+        data = open(os.path.join(bench.ROOT, "token_dispatch_top_b200", "csrc", name)).read()
+        (same / "token_dispatch_top_b200" / "csrc" / name).write_text(data)
+    (same / "profiles").mkdir()
+    rec_same = dict(rec, source_hash=None)
+    monkeypatch.setattr(bench, "ROOT", str(same))
+    rec_same["source_hash"] = bench.kernel_source_hash(rec["source_files"])
+    (same / "profiles" / "traffic.json").write_text(json.dumps(rec_same))
     assert bench.recorded_traffic("k_dispatch") == rec["kernels"]["k_dispatch"][
         "dram_bytes_per_launch"]
-    assert bench.recorded_traffic("k_nothing") is None
+    monkeypatch.undo()
     # a copy of the tree whose kernel source differs: the record no longer applies
     csrc = tmp_path / "token_dispatch_top_b200" / "csrc"
     csrc.mkdir(parents=True)
