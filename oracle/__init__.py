@@ -77,6 +77,14 @@ def _load():
         lib.zbo_dispatch.restype = None
         lib.zbo_combine.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, vp]
         lib.zbo_combine.restype = None
+        lib.zbo_count.argtypes = [ctypes.POINTER(_Cfg), vp, vp]
+        lib.zbo_count.restype = None
+        lib.zbo_plan_rank.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int, _P32, _P32, _P32,
+                                      ctypes.POINTER(_Out)]
+        lib.zbo_dispatch_ranks.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp]
+        lib.zbo_dispatch_ranks.restype = None
+        lib.zbo_combine_ranks.argtypes = [ctypes.POINTER(_Cfg), vp, vp, vp, vp]
+        lib.zbo_combine_ranks.restype = None
         lib.zbo_f32_to_bf16.argtypes = [ctypes.c_float]
         lib.zbo_f32_to_bf16.restype = ctypes.c_uint16
         lib.zbo_bf16_to_f32.argtypes = [ctypes.c_uint16]
@@ -207,6 +215,77 @@ def combine(cfg: Config, dst_row: np.ndarray, y_bits: np.ndarray, w: np.ndarray)
     out = np.zeros((P, S, H), np.uint16)
     _load().zbo_combine(ctypes.byref(cfg.c()), dst_row.ctypes.data, y_bits.ctypes.data,
                         w.ctypes.data, out.ctypes.data)
+    return out
+
+
+def count(cfg: Config, ids_i: np.ndarray) -> np.ndarray:
+    """Step 1 on one rank of a P-rank group: int32 ``[E+1]``, the counts of the
+    rank's own ids ``[S,K]`` per expert, then the number of ids outside
+    [0, E).  These rows are what the ranks exchange."""
+    ids_i = np.ascontiguousarray(ids_i, dtype=np.int32).reshape(cfg.S, cfg.K)
+    row = np.zeros(cfg.E + 1, np.int32)
+    _load().zbo_count(ctypes.byref(cfg.c()), ids_i.ctypes.data, row.ctypes.data)
+    return row
+
+
+def plan_rank(cfg: Config, rank: int, counts: np.ndarray, ids_i: np.ndarray,
+              placement: np.ndarray | None = None) -> dict:
+    """Steps 2-3 as one rank computes them from the exchanged count rows
+    ``counts`` int32 ``[P,E+1]`` and its own ids ``[S,K]``.  Returns the plan
+    tables (as :func:`plan`) with ``dst_row`` ``[S,K]`` for this rank's
+    entries only, and no ``row_src``."""
+    lib = _load()
+    P, E, K, S, R = cfg.P, cfg.E, cfg.K, cfg.S, cfg.R
+    Eh = E // max(P, 1)
+    counts = np.ascontiguousarray(counts, dtype=np.int32).reshape(P, E + 1)
+    ids_i = np.ascontiguousarray(ids_i, dtype=np.int32).reshape(S, K)
+    r = dict(
+        cnt=np.zeros((P, E), np.int32), rep_expert=np.zeros((P, R), np.int32),
+        rep_quota=np.zeros((P, R), np.int32), home_quota=np.zeros(E, np.int32),
+        load_before=np.zeros(P, np.int32), load_after=np.zeros(P, np.int32),
+        cu_seqlens=np.zeros((P, Eh + R + 1), np.int32), dst_row=np.zeros((S, K), np.int32))
+    out = _Out(*[_ptr(r[k]) for k in ("cnt", "rep_expert", "rep_quota", "home_quota",
+                                       "load_before", "load_after", "cu_seqlens", "dst_row")],
+               _P32(), _P32(), 0, 0, 0, 0, 0, 0)
+    pl = None if placement is None else \
+        np.ascontiguousarray(placement, dtype=np.int32).reshape(P, R)
+    st = lib.zbo_plan_rank(ctypes.byref(cfg.c()), int(rank), _ptr(counts), _ptr(ids_i),
+                           _ptr(pl) if pl is not None else _P32(), ctypes.byref(out))
+    r.update(status=int(st), locality_cost=int(out.locality_cost), max_load=int(out.max_load),
+             n_replicas=int(out.n_replicas), n_iters=int(out.n_iters), T=int(out.water_level),
+             repaired=int(out.repaired))
+    return r
+
+
+def _row_pointers(arrays, rows: int, H: int):
+    ptrs = (ctypes.c_void_p * len(arrays))()
+    for j, a in enumerate(arrays):
+        assert a.dtype == np.uint16 and a.flags.c_contiguous and a.shape == (rows, H)
+        ptrs[j] = a.ctypes.data
+    return ptrs
+
+
+def dispatch_ranks(cfg: Config, dst_i: np.ndarray, hidden_i: np.ndarray, bufs) -> None:
+    """Step 4 on one rank: its rows ``hidden_i`` uint16 ``[S,H]`` written into
+    the receive buffers ``bufs`` (P arrays uint16 ``[cap,H]``, one per
+    destination rank) at the rows ``dst_i`` ``[S,K]`` name."""
+    dst_i = np.ascontiguousarray(dst_i, dtype=np.int32).reshape(cfg.S, cfg.K)
+    hidden_i = np.ascontiguousarray(hidden_i, dtype=np.uint16).reshape(cfg.S, cfg.H)
+    ptrs = _row_pointers(bufs, cfg.cap(), cfg.H)
+    _load().zbo_dispatch_ranks(ctypes.byref(cfg.c()), dst_i.ctypes.data, hidden_i.ctypes.data,
+                               ptrs)
+
+
+def combine_ranks(cfg: Config, dst_i: np.ndarray, ys, w_i: np.ndarray) -> np.ndarray:
+    """Step 5 on one rank: uint16 ``[S,H]`` from the expert outputs ``ys`` (P
+    arrays uint16 ``[cap,H]``, one per rank that computed them) and the
+    rank's gates ``w_i`` float32 ``[S,K]``."""
+    dst_i = np.ascontiguousarray(dst_i, dtype=np.int32).reshape(cfg.S, cfg.K)
+    w_i = np.ascontiguousarray(w_i, dtype=np.float32).reshape(cfg.S, cfg.K)
+    ptrs = _row_pointers(ys, cfg.cap(), cfg.H)
+    out = np.zeros((cfg.S, cfg.H), np.uint16)
+    _load().zbo_combine_ranks(ctypes.byref(cfg.c()), dst_i.ctypes.data, ptrs, w_i.ctypes.data,
+                              out.ctypes.data)
     return out
 
 

@@ -503,18 +503,18 @@ int zbo_plan(const zbo_config *c, const int32_t *ids, zbo_plan_out *out) {
   return zbo_plan_placed(c, ids, NULL, out);
 }
 
-/* The whole plan with the replica placement given (placement != NULL: quotas
- * only, by greedy_placed) or chosen by the greedy (placement == NULL). */
-int zbo_plan_placed(const zbo_config *c, const int32_t *ids, const int32_t *placement,
-                    zbo_plan_out *out) {
-  int rc = zbo_validate(c);
-  if (rc) return rc;
-  if (placement && !zbo_placement_valid(c, placement)) return ZBO_ERR_INVALID;
+/* Steps 2-3 from the route counts in out->cnt, which every rank computes
+ * alike once the counts are exchanged [ISER, HALO-Q Scheduler, stage 1]: water
+ * level, greedy placement (placement == NULL) or the kept placement's quotas,
+ * quota repair, transport, cu_seqlens.  Returns ZBO_OK, ZBO_UNBALANCED,
+ * ZBO_ERR_CAPACITY or an error.  Unless it returns an error other than
+ * ZBO_ERR_CAPACITY, *Mall_out holds the transport M[e][i][j] (freed by the
+ * caller). */
+static int plan_from_counts(const zbo_config *c, const int32_t *placement, zbo_plan_out *out,
+                            int32_t **Mall_out) {
   const int P = c->P, E = c->E, R = c->R, Eh = E / P, G = Eh + R;
-  const int64_t NK = (int64_t)c->S * c->K;
-
-  rc = histogram(c, ids, out->cnt);
-  if (rc) return rc;
+  int rc;
+  *Mall_out = NULL;
 
   /* T_e = sum_i cnt[i][e];  L_j = sum over j's home experts of T_e. */
   int32_t *Te = calloc((size_t)E, sizeof(int32_t));
@@ -590,63 +590,198 @@ int zbo_plan_placed(const zbo_config *c, const int32_t *ids, const int32_t *plac
     out->load_after[j] = out->cu_seqlens[(size_t)j * (G + 1) + G];
     if (out->load_after[j] > out->max_load) out->max_load = out->load_after[j];
   }
-  const int64_t cap = c->cap_rows;
-  if (out->row_src)
-    for (int64_t x = 0; x < (int64_t)P * cap; x++) out->row_src[x] = -1;
-  if (out->max_load > c->cap_rows) {
-    for (int64_t x = 0; x < (int64_t)P * NK; x++) out->dst_row[x] = -1;
-    free(Mall); free(Te);
-    return ZBO_ERR_CAPACITY;
-  }
+  free(Te);
+  *Mall_out = Mall;
+  if (out->max_load > c->cap_rows) return ZBO_ERR_CAPACITY;
+  return status;
+}
 
-  /* Rows.  Source i walks its entries of expert e in flat order f = s*K+k
-   * and fills its hosts in order of (a_ij, j): the first M_{i,h1} entries go
-   * to h1, the next M_{i,h2} to h2, ...  Inside host j's group, source i's
-   * segment starts after the rows of sources i' < i. */
+/* The rows of source i.  Source i walks its entries of expert e in flat order
+ * f = s*K+k (ids_i[f]) and fills its hosts in order of (a_ij, j): the first
+ * M_{i,h1} entries go to h1, the next M_{i,h2} to h2, ...  Inside host j's
+ * group, source i's segment starts after the rows of sources i' < i.  Writes
+ * dst_i[f] = j*cap + row, and row_src[j*cap + row] = i*S*K + f when row_src
+ * is not NULL. */
+static void rows_of_source(const zbo_config *c, int i, const int32_t *ids_i,
+                           const int32_t *Mall, const zbo_plan_out *out, int32_t *dst_i,
+                           int32_t *row_src) {
+  const int P = c->P, E = c->E, R = c->R, Eh = E / P, G = Eh + R;
+  const int64_t NK = (int64_t)c->S * c->K;
+  const int64_t cap = c->cap_rows;
   int32_t *cursor = calloc((size_t)E, sizeof(int32_t)); /* index into order */
   int32_t *taken = calloc((size_t)E, sizeof(int32_t));  /* used in current host */
   host_t *hl = malloc(sizeof(host_t) * (size_t)E * 33);
   int *nhl = calloc((size_t)E, sizeof(int));
   for (int e = 0; e < E; e++)
     nhl[e] = hosts_of(c, e, out->home_quota, out->rep_expert, out->rep_quota, hl + (size_t)e * 33);
-  for (int i = 0; i < P; i++) {
-    /* host order of source i for each expert: a ascending, then rank */
-    int32_t *ord = malloc(sizeof(int32_t) * (size_t)E * 33);
-    for (int e = 0; e < E; e++) {
-      int n = 0;
-      for (int a = 0; a <= 4; a++)
-        for (int h = 0; h < nhl[e]; h++)
-          if (cost_a(c, i, hl[(size_t)e * 33 + h].rank) == a) ord[(size_t)e * 33 + n++] = h;
-      cursor[e] = 0;
+  /* host order of source i for each expert: a ascending, then rank */
+  int32_t *ord = malloc(sizeof(int32_t) * (size_t)E * 33);
+  for (int e = 0; e < E; e++) {
+    int n = 0;
+    for (int a = 0; a <= 4; a++)
+      for (int h = 0; h < nhl[e]; h++)
+        if (cost_a(c, i, hl[(size_t)e * 33 + h].rank) == a) ord[(size_t)e * 33 + n++] = h;
+  }
+  for (int64_t f = 0; f < NK; f++) {
+    int e = ids_i[f];
+    int h, j;
+    int32_t Mij;
+    for (;;) {
+      h = ord[(size_t)e * 33 + cursor[e]];
+      j = hl[(size_t)e * 33 + h].rank;
+      Mij = Mall[((size_t)e * P + i) * P + j];
+      if (taken[e] < Mij) break;
+      cursor[e] += 1;
       taken[e] = 0;
     }
-    for (int64_t f = 0; f < NK; f++) {
-      int64_t gidx = (int64_t)i * NK + f;
-      int e = ids[gidx];
-      int h, j;
-      int32_t Mij;
-      for (;;) {
-        h = ord[(size_t)e * 33 + cursor[e]];
-        j = hl[(size_t)e * 33 + h].rank;
-        Mij = Mall[((size_t)e * P + i) * P + j];
-        if (taken[e] < Mij) break;
-        cursor[e] += 1;
-        taken[e] = 0;
-      }
-      int32_t seg = 0;
-      for (int ip = 0; ip < i; ip++) seg += Mall[((size_t)e * P + ip) * P + j];
-      int32_t row = out->cu_seqlens[(size_t)j * (G + 1) + hl[(size_t)e * 33 + h].group] + seg +
-                    taken[e];
-      taken[e] += 1;
-      int32_t dst = (int32_t)(j * cap + row);
-      out->dst_row[gidx] = dst;
-      if (out->row_src) out->row_src[dst] = (int32_t)gidx;
-    }
-    free(ord);
+    int32_t seg = 0;
+    for (int ip = 0; ip < i; ip++) seg += Mall[((size_t)e * P + ip) * P + j];
+    int32_t row = out->cu_seqlens[(size_t)j * (G + 1) + hl[(size_t)e * 33 + h].group] + seg +
+                  taken[e];
+    taken[e] += 1;
+    int32_t dst = (int32_t)(j * cap + row);
+    dst_i[f] = dst;
+    if (row_src) row_src[dst] = (int32_t)((int64_t)i * NK + f);
   }
-  free(nhl); free(hl); free(taken); free(cursor);
-  free(Mall); free(Te);
+  free(ord); free(nhl); free(hl); free(taken); free(cursor);
+}
+
+/* The whole plan with the replica placement given (placement != NULL: quotas
+ * only, by greedy_placed) or chosen by the greedy (placement == NULL). */
+int zbo_plan_placed(const zbo_config *c, const int32_t *ids, const int32_t *placement,
+                    zbo_plan_out *out) {
+  int rc = zbo_validate(c);
+  if (rc) return rc;
+  if (placement && !zbo_placement_valid(c, placement)) return ZBO_ERR_INVALID;
+  const int P = c->P;
+  const int64_t NK = (int64_t)c->S * c->K;
+
+  rc = histogram(c, ids, out->cnt);
+  if (rc) return rc;
+
+  int32_t *Mall;
+  int status = plan_from_counts(c, placement, out, &Mall);
+  if (status < 0 && status != ZBO_ERR_CAPACITY) return status;
+  if (out->row_src)
+    for (int64_t x = 0; x < (int64_t)P * c->cap_rows; x++) out->row_src[x] = -1;
+  if (status == ZBO_ERR_CAPACITY) {
+    for (int64_t x = 0; x < (int64_t)P * NK; x++) out->dst_row[x] = -1;
+    free(Mall);
+    return status;
+  }
+  for (int i = 0; i < P; i++)
+    rows_of_source(c, i, ids + (int64_t)i * NK, Mall, out, out->dst_row + (int64_t)i * NK,
+                   out->row_src);
+  free(Mall);
   return status;
+}
+
+/* ------------------------------------------- the path on one of P ranks */
+
+/* Step 1 on one rank of a P-rank group: the route counts of the rank's own
+ * entries ids_i[f], f < S*K: row[e] = #{f : ids_i[f] = e} for e < E, and
+ * row[E] = the number of ids outside [0, E).  These rows are what the ranks
+ * exchange before planning [ISER, HALO-Q Scheduler, stage 1: ranks share their
+ * route counts through a symmetric NVLink buffer]. */
+void zbo_count(const zbo_config *c, const int32_t *ids_i, int32_t *row) {
+  memset(row, 0, sizeof(int32_t) * (size_t)(c->E + 1));
+  for (int64_t f = 0; f < (int64_t)c->S * c->K; f++) {
+    int32_t e = ids_i[f];
+    if (e < 0 || e >= c->E)
+      row[c->E] += 1;
+    else
+      row[e] += 1;
+  }
+}
+
+/* Steps 2-3 as rank `rank` computes them when it holds only its own ids
+ * ids_i [S][K] and the exchanged count rows counts [P][E+1] (zbo_count of
+ * every rank, in rank order).  The tables depend on the counts alone, so
+ * every rank computes the same ones; the rows of the rank's own entries
+ * depend on the counts and its own ids [ISER, HALO-Q Scheduler: stage 1
+ * exchanges the counts, and every rank then plans]. out->dst_row is [S][K]
+ * (this rank's entries); out->row_src is not written.
+ * Returns as zbo_plan_placed, and ZBO_ERR_INVALID when counts[rank] is not the
+ * count of ids_i or a row does not sum to S*K; ZBO_ERR_BAD_ID when any rank
+ * counted an id outside [0, E). */
+int zbo_plan_rank(const zbo_config *c, int rank, const int32_t *counts, const int32_t *ids_i,
+                  const int32_t *placement, zbo_plan_out *out) {
+  int rc = zbo_validate(c);
+  if (rc) return rc;
+  if (rank < 0 || rank >= c->P) return ZBO_ERR_INVALID;
+  if (placement && !zbo_placement_valid(c, placement)) return ZBO_ERR_INVALID;
+  const int P = c->P, E = c->E;
+  const int64_t NK = (int64_t)c->S * c->K;
+
+  int32_t *mine = calloc((size_t)E + 1, sizeof(int32_t));
+  zbo_count(c, ids_i, mine);
+  int same = memcmp(mine, counts + (size_t)rank * (E + 1), sizeof(int32_t) * (size_t)(E + 1)) == 0;
+  free(mine);
+  if (!same) return ZBO_ERR_INVALID;
+  int64_t bad = 0;
+  for (int i = 0; i < P; i++) {
+    int64_t sum = 0;
+    for (int e = 0; e <= E; e++) {
+      int32_t v = counts[(size_t)i * (E + 1) + e];
+      if (v < 0) return ZBO_ERR_INVALID;
+      sum += v;
+    }
+    if (sum != NK) return ZBO_ERR_INVALID;
+    bad += counts[(size_t)i * (E + 1) + E];
+  }
+  if (bad) return ZBO_ERR_BAD_ID;
+  for (int i = 0; i < P; i++)
+    for (int e = 0; e < E; e++) out->cnt[(size_t)i * E + e] = counts[(size_t)i * (E + 1) + e];
+
+  int32_t *Mall;
+  int status = plan_from_counts(c, placement, out, &Mall);
+  if (status < 0 && status != ZBO_ERR_CAPACITY) return status;
+  if (status == ZBO_ERR_CAPACITY) {
+    for (int64_t f = 0; f < NK; f++) out->dst_row[f] = -1;
+    free(Mall);
+    return status;
+  }
+  rows_of_source(c, rank, ids_i, Mall, out, out->dst_row, NULL);
+  free(Mall);
+  return status;
+}
+
+/* Step 4 on one rank: its token rows written straight into the fixed-shape,
+ * expert-grouped receive buffers of their destination ranks [MOON, "What
+ * MoonEP enforces and how": zero-copy writes into buffers on remote ranks].
+ * bufs[j] is rank j's buffer [cap][H].  For each entry f = s*K+k with
+ * d = dst_i[f] >= 0: bufs[d / cap][d % cap] = hidden_i[s]. */
+void zbo_dispatch_ranks(const zbo_config *c, const int32_t *dst_i, const uint16_t *hidden_i,
+                        uint16_t *const *bufs) {
+  const int64_t H = c->H, cap = c->cap_rows;
+  for (int64_t s = 0; s < c->S; s++)
+    for (int k = 0; k < c->K; k++) {
+      int32_t d = dst_i[s * c->K + k];
+      if (d < 0) continue;
+      memcpy(bufs[d / cap] + (d % cap) * H, hidden_i + s * H, sizeof(uint16_t) * (size_t)H);
+    }
+}
+
+float zbo_bf16_to_f32(uint16_t b);
+uint16_t zbo_f32_to_bf16(float f);
+
+/* Step 5 on one rank: each of its tokens gathers its K expert outputs from the
+ * ranks that computed them, ys[j] being rank j's rows [cap][H]:
+ *   acc = +0.0f; acc = fmaf(w_i[s,k], ys[d / cap][d % cap][h], acc) for
+ *   k = 0..K-1 with d = dst_i[s*K+k]; out_i[s][h] = bf16(acc),
+ * the same fold and rounding as zbo_combine. */
+void zbo_combine_ranks(const zbo_config *c, const int32_t *dst_i, const uint16_t *const *ys,
+                       const float *w_i, uint16_t *out_i) {
+  const int64_t H = c->H, cap = c->cap_rows;
+  for (int64_t s = 0; s < c->S; s++)
+    for (int64_t h = 0; h < H; h++) {
+      float acc = 0.0f;
+      for (int k = 0; k < c->K; k++) {
+        int64_t d = dst_i[s * c->K + k];
+        acc = fmaf(w_i[s * c->K + k], zbo_bf16_to_f32(ys[d / cap][(d % cap) * H + h]), acc);
+      }
+      out_i[s * H + h] = zbo_f32_to_bf16(acc);
+    }
 }
 
 /* -------------------------------------- placement from historical demand */
