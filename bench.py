@@ -1,18 +1,22 @@
 """Benchmark: plan + dispatch + combine tokens/s on B200, with the HBM roofline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload tiny|mid|hot|hier|drift] [--no-extras]
 
 One step is one invocation of the whole hot path (histogram, greedy replica
-plan, assignment, dispatch scatter, combine gather) on the mid workload: P=8
-virtual ranks, E=64, K=6, S=4096 tokens per rank, H=2048 bf16, R=2, C=0.1,
-Zipf s=1.2 popularity with a per-seed permuted ranking.  The expert outputs fed
-to the combine are the dispatched rows themselves (identity experts), so the
-step moves exactly the dispatch and combine traffic.
+plan, assignment, dispatch scatter, combine gather) on the headline workload,
+by default mid: P=8 virtual ranks, E=64, K=6, S=4096 tokens per rank, H=2048
+bf16, R=2, C=0.1, Zipf s=1.2 popularity with a per-seed permuted ranking.  The
+expert outputs fed to the combine are the dispatched rows themselves
+(identity experts), so the step moves exactly the dispatch and combine
+traffic.  Inputs are seeded and synthetic.
 
 * ``value``: tokens/s over all ranks, device-timed with CUDA events with the
-  inputs resident in HBM; L2 (126 MB) is flushed before every step, outside
-  the timed events, by a 256 MB write followed by a 256 MB read (so no dirty
-  flush lines are written back inside the timed step).
+  inputs resident in HBM, steps pipelined two deep (the plan of step k+1 on
+  its own stream beside the rows of step k).  Every step streams its rows
+  through buffers larger than L2.
+* ``serial``: the same steps one at a time, L2 flushed before each (outside
+  the events) by a 256 MB write and a 256 MB read; per-kernel event times.
 * ``e2e``: the same metric through the public API with pinned host buffers:
   each step copies ids, weights and hidden rows host->device, runs the path,
   and copies the combined rows and the plan status back; the copies run on
@@ -22,12 +26,14 @@ step moves exactly the dispatch and combine traffic.
   event-timed duration, against the measured HBM copy bandwidth.
 * ``cpu_baseline``: the CPU oracle (single thread) on full steps of the same
   workload, rank 0 at N=1 only.
+* ``extras.workloads`` (N=1): the other four workloads one invocation at a
+  time: plan latency, dispatch and combine rates and fractions of the peak,
+  and the plan's balance (drift: steps 0, 31 and 63).
 
 With ``--impl reference`` the CPU oracle itself is timed on the same workload
 (rank 0 only; other ranks exit).  With N>1 (torchrun), every rank runs an
-independent replica on its own GPU (the path has no cross-rank exchange on one
-GPU); ``value`` is the sum of tokens over ranks divided by the slowest rank's
-time.
+independent replica on its own GPU; ``value`` is the sum of tokens over ranks
+divided by the slowest rank's time.
 """
 from __future__ import annotations
 
@@ -54,8 +60,33 @@ FALLBACK_HBM_GBS = 6650.0
 
 
 def workload_desc(wl) -> str:
-    return (f"{wl.name}: P={wl.P} E={wl.E} K={wl.K} S={wl.S} H={wl.H} R={wl.R} C={wl.C}, "
-            f"Zipf s={wl.zipf_s} popularity, permuted ranking, seed 0")
+    if wl.hot_share is not None:
+        pop = (f"4 hottest experts take {wl.hot_share:.0%} of assignments, the rest Zipf "
+               f"s={wl.hot_zipf_s}")
+    else:
+        pop = f"Zipf s={wl.zipf_s} popularity"
+    if wl.permute:
+        pop += ", permuted ranking"
+    if wl.walk_sigma:
+        pop += f", log-popularity random walk sigma={wl.walk_sigma} per step"
+    nodes = f", {wl.P // wl.gpus_per_node} nodes x {wl.gpus_per_node}" \
+        if wl.gpus_per_node > 1 else ""
+    return (f"{wl.name}: P={wl.P}{nodes} E={wl.E} K={wl.K} S={wl.S} H={wl.H} R={wl.R} "
+            f"C={wl.C}, {pop}, seed 0")
+
+
+def config_dict(wl, n_gpus: int) -> dict:
+    """The ``config`` both arms print for a workload (identical keys and text)."""
+    return {"workload": workload_desc(wl), "tokens_per_step_per_gpu": wl.tokens,
+            "l2": "the timed loop streams every step's rows through buffers larger than "
+                  "L2 (126 MB); the serial loop also flushes L2 before each step",
+            "parallelism": f"replicas x{n_gpus}"}
+
+
+def data_cap_rows(wl) -> int | None:
+    """Receive-buffer rows: the water level S*K for the workloads that balance
+    (tiny, mid); twice that for the ones whose slots cannot reach it."""
+    return None if wl.name in ("tiny", "mid") else 2 * wl.S * wl.K
 
 
 def algorithmic_bytes(wl) -> dict:
@@ -219,7 +250,8 @@ def run_reference(args, wl, rank, budget_s: float = 120.0):
     from token_dispatch_top_b200 import synth
     ids, w = synth.routing(wl, 0)
     hidden = synth.hidden_bits(wl, 0)
-    cfg = oracle.Config(wl.P, wl.E, wl.K, wl.S, wl.H, wl.R, wl.C, wl.gpus_per_node, None)
+    cfg = oracle.Config(wl.P, wl.E, wl.K, wl.S, wl.H, wl.R, wl.C, wl.gpus_per_node,
+                        data_cap_rows(wl))
     buf = np.empty((wl.P, cfg.cap(), wl.H), np.uint16)
     probe = min(1024, wl.tokens)
     tp, td = oracle_sampled_step(wl, cfg, ids, w, hidden, buf, probe)
@@ -239,7 +271,7 @@ def run_reference(args, wl, rank, budget_s: float = 120.0):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * full_step_s, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": workload_desc(wl), "tokens_per_step": wl.tokens},
+        "config": config_dict(wl, args.gpus),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": f"per step: the full plan plus dispatch and combine of "
                                    f"{n_tok} of {wl.tokens} tokens, scaled to all tokens; "
@@ -248,6 +280,70 @@ def run_reference(args, wl, rank, budget_s: float = 120.0):
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def measure_workload(wl, dev, flush_l2, peak, iters=10, steps=(0,)):
+    """One workload's kernels, one invocation at a time (L2 flushed before
+    each, outside the events): plan, dispatch and combine times, their HBM
+    rates against the measured peak, and the plan's balance.  Drift steps
+    rotate through ``steps``, each with its own ids and gates."""
+    import torch
+    from token_dispatch_top_b200 import metrics, synth, zb
+    cfg = zb.Config(P=wl.P, E=wl.E, K=wl.K, S=wl.S, H=wl.H, R=wl.R, C=wl.C,
+                    gpus_per_node=wl.gpus_per_node, cap_rows=data_cap_rows(wl))
+    P, S, H, cap = cfg.P, cfg.S, cfg.H, cfg.cap
+    inputs = []
+    for st in steps:
+        ids_np, w_np = synth.routing(wl, 0, st)
+        inputs.append((torch.from_numpy(ids_np).to(dev), torch.from_numpy(w_np).to(dev)))
+    hidden = synth.hidden_device(wl, 0, 0, dev)
+    plan = zb.Plan(cfg, dev, with_row_src=False)
+    buf = torch.empty((P, cap, H), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((P, S, H), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    t_plan, t_disp, t_comb, balance = [], [], [], []
+    for it in range(3 + iters):
+        ids, w = inputs[it % len(inputs)]
+        flush_l2()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
+        zb.plan(plan, ids)
+        ev[1].record(stream)
+        zb.dispatch(plan, hidden, buf)
+        ev[2].record(stream)
+        zb.combine(plan, buf, w, out)
+        ev[3].record(stream)
+        status, _ = zb.plan_status(plan)
+        if status < 0:
+            raise RuntimeError(f"{wl.name}: plan failed: {zb.strerror(status)}")
+        if it >= 3:
+            t_plan.append(ev[0].elapsed_time(ev[1]))
+            t_disp.append(ev[1].elapsed_time(ev[2]))
+            t_comb.append(ev[2].elapsed_time(ev[3]))
+        if it < len(inputs):
+            m = metrics.plan_metrics(plan)
+            balance.append({"step": steps[it], "status": status,
+                            "r_imb_before": m["r_imb_before"], "r_imb_after": m["r_imb_after"],
+                            "max_load_over_T": int(plan.stats[zb.STAT_MAX_LOAD]) /
+                            max(1, int(plan.stats[zb.STAT_WATER_LEVEL]))})
+    ab = algorithmic_bytes(wl)
+    d, c, pl = (statistics.median(t_disp), statistics.median(t_comb),
+                statistics.median(t_plan))
+    rec = {"workload": workload_desc(wl), "cap_rows": cap, "steps": list(steps),
+           "iterations": iters, "plan_us": 1000.0 * pl,
+           "dispatch": {"ms": d, "gbs": ab["dispatch"] / d / 1e6,
+                        "frac": ab["dispatch"] / d / 1e6 / peak,
+                        "algorithmic_bytes": ab["dispatch"]},
+           "combine": {"ms": c, "gbs": ab["combine"] / c / 1e6,
+                       "frac": ab["combine"] / c / 1e6 / peak,
+                       "algorithmic_bytes": ab["combine"],
+                       "kernel": "k_combine_wide (32-byte loads)"
+                       if wl.K in (7, 8) and wl.H >= 4096 else "k_combine"},
+           "tokens_per_s": wl.tokens / ((pl + d + c) / 1000.0),
+           "balance": balance}
+    del plan, buf, out, hidden, inputs
+    torch.cuda.empty_cache()
+    return rec
 
 
 def run_ours(args, wl, rank, world, local_rank):
@@ -267,7 +363,7 @@ def run_ours(args, wl, rank, world, local_rank):
     ids_np, w_np = synth.routing(wl, seed)
     hidden_np = synth.hidden_bits(wl, seed)
     cfg = zb.Config(P=wl.P, E=wl.E, K=wl.K, S=wl.S, H=wl.H, R=wl.R, C=wl.C,
-                    gpus_per_node=wl.gpus_per_node)
+                    gpus_per_node=wl.gpus_per_node, cap_rows=data_cap_rows(wl))
     P, S, K, H, cap = cfg.P, cfg.S, cfg.K, cfg.H, cfg.cap
 
     ids = torch.from_numpy(ids_np).to(dev)
@@ -563,6 +659,19 @@ def run_ours(args, wl, rank, world, local_rank):
     h2d = ids_np.nbytes + w_np.nbytes + hidden_np.nbytes
     d2h = P * S * H * 2 + zb.STATS_LEN * 8
 
+    # ---- the other workloads, one invocation at a time (N = 1 only): plan
+    # latency, dispatch and combine rates, balance
+    workloads = {}
+    if world == 1 and args.extras:
+        peak_gbs, _ = read_peaks()
+        torch.cuda.empty_cache()
+        for name in ("tiny", "mid", "hot", "hier", "drift"):
+            if name == wl.name:
+                continue
+            steps = (0, 31, 63) if name == "drift" else (0,)
+            workloads[name] = measure_workload(synth.WORKLOADS[name], dev, flush_l2, peak_gbs,
+                                               steps=steps)
+
     # ---- max over ranks
     (step_ms, e2e_ms, disp_ms, comb_ms, plan_ms, serial_ms, s_disp_ms, s_comb_ms,
      s_plan_ms) = max_over_ranks(
@@ -595,15 +704,14 @@ def run_ours(args, wl, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": workload_desc(wl), "tokens_per_step_per_gpu": wl.tokens,
-                   "accumulate": "f32", "experts": "identity (y = dispatched rows)",
+        "config": config_dict(wl, world),
+        "method": {"accumulate": "f32", "experts": "identity (y = dispatched rows)",
                    "pipeline": "two steps in flight: the plan of step k+1 runs on a "
                                "high-priority stream while the rows of step k move; two "
                                "slots of plan, receive and output buffers",
-                   "l2": "not flushed in the timed (pipelined) loop: every step streams "
-                         "1.9 GB through buffers larger than L2 (hidden 134 MB, receive "
-                         "buffers 805 MB); the serial loop flushes before every step",
-                   "parallelism": f"replicas x{world}"},
+                   "l2": f"not flushed in the timed (pipelined) loop: every step streams "
+                         f"{sum(algorithmic_bytes(wl).values()) / 1e9:.2f} GB through buffers "
+                         f"larger than L2; the serial loop flushes before every step"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "method": "pinned host buffers; per step H2D of ids, gates and hidden, "
@@ -644,7 +752,10 @@ def run_ours(args, wl, rank, world, local_rank):
                 "combine_ms": statistics.median(cm_ms),
                 "combine_gbs": (rows_merged * wl.H * 2 + wl.N * 4 + wl.tokens * wl.H * 2)
                 / statistics.median(cm_ms) / 1e6},
-            "banded_plan": banded, "quota_repair": rep},
+            "banded_plan": banded, "quota_repair": rep,
+            "workloads": workloads},
+        "plan_latency_us": dict({wl.name: 1000.0 * s_plan_ms / args.steps},
+                                **{k: v["plan_us"] for k, v in workloads.items()}),
         "wall_s": wall,
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,
@@ -658,6 +769,10 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["tiny", "mid", "hot", "hier", "drift"],
+                    default=WORKLOAD, help="the headline workload (default: mid)")
+    ap.add_argument("--no-extras", dest="extras", action="store_false",
+                    help="skip the per-workload records of the other workloads")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be at least 3")
@@ -666,7 +781,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     from token_dispatch_top_b200 import synth
-    wl = synth.WORKLOADS[WORKLOAD]
+    wl = synth.WORKLOADS[args.workload]
 
     if args.impl == "reference":
         run_reference(args, wl, rank)

@@ -1,7 +1,9 @@
 /*
- * zb.h -- C ABI of libzb: load-balanced MoE token dispatch and combine on one
- * B200 (sm_100a), with the P expert-parallel ranks virtual and their buffers
- * partitioned inside one device memory.
+ * zb.h -- C ABI of libzb: load-balanced MoE token dispatch and combine on
+ * B200 (sm_100a) across P expert-parallel ranks: virtual ranks whose buffers
+ * partition one device memory (zb_plan, zb_dispatch, zb_combine), or one rank
+ * per GPU, each holding its own tokens (zb_count, zb_plan_rank,
+ * zb_dispatch_rank, zb_combine_rank).
  *
  * One invocation is five steps, in order:
  *   1. per-rank, per-expert histogram of the top-K routing ids        (zb_plan)
@@ -11,9 +13,13 @@
  *   5. gate-weighted combine gather, fp32 accumulation in k order     (zb_combine)
  *
  * Conventions for every entry point:
- *  - Every pointer argument except `cfg`, `plan` (the struct itself) and the
- *    out-parameters of zb_plan_status is DEVICE memory owned by the caller.
- *    The library allocates nothing and keeps no state between calls.
+ *  - Every pointer argument is DEVICE memory owned by the caller, except
+ *    `cfg`, the `plan` and `merge` structs themselves, the host out-parameters
+ *    of zb_plan_status and zb_recalibrate, the host arrays of zb_place_by_demand,
+ *    and the host tables of per-rank device pointers taken by
+ *    zb_dispatch_rank and zb_combine_rank.  The library allocates nothing and
+ *    keeps no state between calls (zb_plan_noalloc's fixed scratch array is
+ *    the one exception, described there).
  *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *    stream).  Every call except zb_plan_status only enqueues work on it and
  *    returns without synchronising.
@@ -247,8 +253,11 @@ ZB_API int zb_plan_status(const zb_config *cfg, const zb_plan_t *plan, void *str
  *    zb_plan gives).
  *  - The scratch belongs to the calling thread's current device, so `stream`
  *    must belong to that device too.  The first call on a device looks up the
- *    array's device address (once per device) and caches it; make that first
- *    call before any stream capture starts.
+ *    array's device address (once per device) and caches it for the life of
+ *    the process; make that first call before any stream capture starts.  A
+ *    process that resets a device (cudaDeviceReset) must not call
+ *    zb_plan_noalloc on that device again: the library's module is loaded
+ *    anew and the cached address no longer names the array.
  *  - Every call on a device shares the one array, which keeps what the last
  *    call left in it; each call clears what it needs zeroed.  Calls whose work
  *    overlaps on the GPU (two streams, or two host threads) race on the
@@ -279,6 +288,83 @@ ZB_API int zb_dispatch(const zb_config *cfg, const zb_plan_t *plan, const uint16
  * ZB_OK, ZB_ERR_INVALID or ZB_ERR_CUDA. */
 ZB_API int zb_combine(const zb_config *cfg, const zb_plan_t *plan, const uint16_t *y,
                const float *topk_weights, uint16_t *out, void *stream);
+
+/* ------------------------------------------- the path on one of P GPUs */
+
+/* The same five steps when the P ranks are P GPUs, one process (or thread)
+ * per GPU, each holding only its own S tokens: ISER-MoE ("Methodology /
+ * HALO-Q Scheduler", stage 1) has the ranks exchange their route counts and
+ * then every rank plan alike; MoonEP ("What MoonEP enforces and how") has
+ * each rank write its rows straight into the fixed-shape, expert-grouped
+ * receive buffers of the other ranks.  On rank i:
+ *   1. zb_count: the counts of its own ids (one row of E+1 ints);
+ *   2. the caller all-gathers every rank's row, in rank order, into a
+ *      [P][E+1] table (for example an NCCL all-gather of P*(E+1) int32);
+ *   3. zb_plan_rank: the plan from that table, identical on every rank,
+ *      and the destination rows of its own entries;
+ *   4. zb_dispatch_rank: its rows written into every rank's receive buffer;
+ *   5. after the expert computation, zb_combine_rank: its tokens' outputs
+ *      gathered from every rank's expert output buffer.
+ * Between 4 and the expert computation, and between the expert computation
+ * and 5, the ranks must synchronise (for example a barrier on the stream):
+ * these calls only move rows and never wait for another rank.
+ *
+ * For rank i, every table these calls produce equals zb_plan's over the whole
+ * batch, and plan->dst_row [S][K] equals zb_plan's rows of source i (values
+ * j*cap + row, as there).  On one GPU the P buffers may be P parts of one
+ * allocation, which reproduces zb_dispatch and zb_combine bit for bit. */
+
+/* Bytes of device scratch memory zb_count and zb_plan_rank need (0 if cfg
+ * is invalid): the per-chunk histograms of this rank's ids and the segment
+ * table. */
+ZB_API size_t zb_rank_workspace_bytes(const zb_config *cfg);
+
+/* Step 1 on one rank: counts[e] = #{(s,k) : ids[s][k] = e} for e < E and
+ * counts[E] = the number of ids outside [0, E).  ids: device int32 [S][K],
+ * this rank's entries; counts: device int32 [E+1]; workspace:
+ * zb_rank_workspace_bytes(cfg) bytes, 256-byte aligned.  The workspace keeps
+ * the per-chunk histograms that zb_plan_rank reads: pass the same workspace,
+ * untouched, and the same ids to the zb_plan_rank that follows.  Returns
+ * ZB_OK, ZB_ERR_INVALID or ZB_ERR_CUDA. */
+ZB_API int zb_count(const zb_config *cfg, const int32_t *topk_ids, int32_t *counts,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/* Steps 2-3 on rank `rank` (0 <= rank < P): counts is the all-gathered
+ * device table int32 [P][E+1] (rank j's zb_count row at j), topk_ids this
+ * rank's ids [S][K], placement NULL (the greedy places the replicas) or a
+ * kept placement as for zb_plan_placed.  plan: as for zb_plan, except that
+ * dst_row is [S][K] (this rank's entries) and row_src must be NULL.
+ * workspace: the one zb_count filled for these ids.  The plan's status
+ * (zb_plan_status) is ZB_ERR_INVALID when counts[rank] is not the count of
+ * this rank's ids or a row of counts does not hold S*K non-negative counts,
+ * and ZB_ERR_BAD_ID on every rank when any rank counted an id outside
+ * [0, E); otherwise as zb_plan.  Returns ZB_OK once enqueued, ZB_ERR_INVALID
+ * or ZB_ERR_CUDA. */
+ZB_API int zb_plan_rank(const zb_config *cfg, int rank, const int32_t *counts,
+                        const int32_t *topk_ids, const int32_t *placement, const zb_plan_t *plan,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/* Step 4 on one rank: for each entry (s,k) of this rank with
+ * d = plan->dst_row[s][k], bufs[d / cap][d % cap][:] = hidden[s][:], bit for
+ * bit.  bufs is a HOST array of P device pointers, bufs[j] = rank j's receive
+ * buffer bf16 [cap][H], 16-byte aligned: peer memory mapped into this process
+ * (CUDA IPC or symmetric memory) for the other ranks, or P parts of one
+ * buffer on one GPU.  Rows go out as plain stores.  hidden: device bf16
+ * [S][H], this rank's rows.  If the plan's status is an error nothing is
+ * written.  Returns ZB_OK, ZB_ERR_INVALID or ZB_ERR_CUDA. */
+ZB_API int zb_dispatch_rank(const zb_config *cfg, const zb_plan_t *plan, const uint16_t *hidden,
+                            uint16_t *const *bufs, void *stream);
+
+/* Step 5 on one rank: for each token s of this rank,
+ *   acc = +0.0f; acc = fmaf(w[s][k], float(ys[d/cap][d%cap][h]), acc) for
+ *   k = 0..K-1, d = plan->dst_row[s][k]; out[s][h] = bf16(acc), nearest even,
+ * the fold of zb_combine.  ys: HOST array of P device pointers, ys[j] = rank
+ * j's expert outputs bf16 [cap][H] in its receive buffer's rows, 16-byte
+ * aligned (read with plain loads); topk_weights: device float32 [S][K]; out:
+ * device bf16 [S][H].  If the plan's status is an error nothing is written.
+ * Returns ZB_OK, ZB_ERR_INVALID or ZB_ERR_CUDA. */
+ZB_API int zb_combine_rank(const zb_config *cfg, const zb_plan_t *plan, const uint16_t *const *ys,
+                           const float *topk_weights, uint16_t *out, void *stream);
 
 /* ------------------------------------------------------- merged dispatch */
 

@@ -102,3 +102,45 @@ def test_entry_points_reject_bad_arguments_without_a_device(lib):
         zb.ERR_INVALID
     assert lib.zb_plan(ctypes.byref(cfg), 16, ctypes.byref(fake), 128, ws, None) == \
         zb.ERR_INVALID
+
+
+def test_rank_entry_points_reject_bad_arguments_without_a_device(lib):
+    """The per-rank form (one rank of P GPUs): workspace sizing and argument
+    checks, all refused before anything is enqueued."""
+    zc = zb.Config(P=4, E=16, K=2, S=64, H=128, R=1)
+    cfg = zc.c()
+    n = lib.zb_rank_workspace_bytes(ctypes.byref(cfg))
+    assert 0 < n < zb.workspace_bytes(zc) and n % 256 == 0  # one source's histograms
+    bad = zb.Config(P=4, E=15, K=2, S=64, H=128, R=1).c()
+    assert lib.zb_rank_workspace_bytes(ctypes.byref(bad)) == 0
+    fake = zb._Plan(*([16] * 10))
+    fake.row_src = None
+    # zb_count: NULL counts, short or misaligned workspace
+    assert lib.zb_count(ctypes.byref(cfg), 16, None, 256, n, None) == zb.ERR_INVALID
+    assert lib.zb_count(ctypes.byref(cfg), 16, 16, 256, n - 1, None) == zb.ERR_INVALID
+    assert lib.zb_count(ctypes.byref(cfg), 16, 16, 128, n, None) == zb.ERR_INVALID
+    # zb_plan_rank: rank out of range, row_src given, NULL counts
+    for rank in (-1, 4):
+        assert lib.zb_plan_rank(ctypes.byref(cfg), rank, 16, 16, None, ctypes.byref(fake), 256,
+                                n, None) == zb.ERR_INVALID
+    with_row_src = zb._Plan(*([16] * 10))
+    assert lib.zb_plan_rank(ctypes.byref(cfg), 0, 16, 16, None, ctypes.byref(with_row_src), 256,
+                            n, None) == zb.ERR_INVALID
+    assert lib.zb_plan_rank(ctypes.byref(cfg), 0, None, 16, None, ctypes.byref(fake), 256, n,
+                            None) == zb.ERR_INVALID
+    # dispatch / combine through a pointer table: a NULL or misaligned entry
+    tbl = (ctypes.c_void_p * 4)(16, 32, 48, 64)
+    holes = (ctypes.c_void_p * 4)(16, None, 48, 64)
+    skew = (ctypes.c_void_p * 4)(16, 40, 48, 64)
+    assert lib.zb_dispatch_rank(ctypes.byref(cfg), ctypes.byref(fake), 16, holes, None) == \
+        zb.ERR_INVALID
+    assert lib.zb_dispatch_rank(ctypes.byref(cfg), ctypes.byref(fake), 16, skew, None) == \
+        zb.ERR_INVALID
+    assert lib.zb_dispatch_rank(ctypes.byref(cfg), ctypes.byref(fake), 8, tbl, None) == \
+        zb.ERR_INVALID
+    assert lib.zb_dispatch_rank(ctypes.byref(cfg), ctypes.byref(fake), 16, None, None) == \
+        zb.ERR_INVALID
+    assert lib.zb_combine_rank(ctypes.byref(cfg), ctypes.byref(fake), holes, 16, 16, None) == \
+        zb.ERR_INVALID
+    assert lib.zb_combine_rank(ctypes.byref(cfg), ctypes.byref(fake), tbl, 16, 8, None) == \
+        zb.ERR_INVALID

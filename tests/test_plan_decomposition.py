@@ -9,6 +9,9 @@ without exchanging their ids (the P-GPU form of the path).
   own ids, all-gathers the count rows, fills the other ranks' entries with
   any ids of the same counts, plans, and gets exactly the global plan's rows
   for its own source.
+* The same protocol through the library binding's count exchange
+  (``zb.exchange_counts``) and the oracle's per-rank plan: each rank's
+  tables and rows equal the global plan's, under every option.
 """
 import os
 import socket
@@ -106,3 +109,59 @@ def test_count_exchange_protocol_gloo(seed):
     for r in range(world):
         np.testing.assert_array_equal(got[r][0], ref["dst_row"][r])
         np.testing.assert_array_equal(got[r][1], ref["cu_seqlens"])
+
+
+def _rank_main_binding(rank, world, port, seed, opts, q):
+    import torch
+    import torch.distributed as dist
+    from token_dispatch_top_b200 import zb
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        cfg, ids = _case(seed, P=world, **opts)
+        mine = torch.from_numpy(oracle.count(cfg, ids[rank]))  # only this rank's ids
+        table = torch.empty((world, cfg.E + 1), dtype=torch.int32)
+        zb.exchange_counts(mine, table)
+        p = oracle.plan_rank(cfg, rank, table.numpy(), ids[rank])
+        q.put((rank, p["status"], p["dst_row"].copy(), {k: p[k].copy() for k in TABLES}))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("seed,opts", [(5, {}), (6, dict(policy=1, relax=1)),
+                                       (7, dict(repair=1, R=3))])
+def test_binding_count_exchange_gloo(seed, opts):
+    world = 4
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main_binding, args=(r, world, port, seed, opts, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = dict()
+    for _ in range(world):
+        r, st, rows, tables = q.get(timeout=120)
+        got[r] = (st, rows, tables)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    cfg, ids = _case(seed, P=world, **opts)
+    ref = oracle.plan(cfg, ids, want_M=False)
+    for r in range(world):
+        st, rows, tables = got[r]
+        assert st == ref["status"]
+        np.testing.assert_array_equal(rows, ref["dst_row"][r])
+        for k in TABLES:
+            np.testing.assert_array_equal(tables[k], ref[k], err_msg=k)
+
+
+def test_exchange_without_a_process_group():
+    import torch
+    from token_dispatch_top_b200 import zb
+    row = torch.arange(5, dtype=torch.int32)
+    table = torch.empty((1, 5), dtype=torch.int32)
+    zb.exchange_counts(row, table)
+    assert torch.equal(table[0], row)
+    with pytest.raises(zb.ZbError):
+        zb.exchange_counts(row, torch.empty((2, 5), dtype=torch.int32))

@@ -57,6 +57,46 @@ def test_noalloc_matches_zb_plan_on_two_calls(lib, cuda_device):
             assert torch.equal(getattr(mine, t), getattr(ref, t)), (seed, t)
 
 
+def _compare_with_zb_plan(lib, cfg, ids, dev):
+    ref = zb.Plan(cfg, dev)
+    zb.plan(ref, ids)
+    mine = zb.Plan(cfg, dev)
+    for t in TABLES:
+        getattr(mine, t).fill_(-7)
+    assert _noalloc(lib, mine, ids) == zb.OK
+    assert zb.plan_status(mine) == zb.plan_status(ref)
+    for t in TABLES:
+        assert torch.equal(getattr(mine, t), getattr(ref, t)), t
+
+
+def test_noalloc_band_and_repair(lib, cuda_device):
+    """The options that use the most planner state: eq. (1)'s band and quota
+    repair, the band's larger receive buffers included."""
+    wl = synth.WORKLOADS["mid"]
+    cfg = zb.Config(P=wl.P, E=wl.E, K=wl.K, S=wl.S, H=wl.H, R=wl.R, C=wl.C, relax=1, repair=1,
+                    policy=zb.POLICY_LOCAL)
+    ids_np, _ = synth.routing(wl, 2)
+    _compare_with_zb_plan(lib, cfg, torch.from_numpy(ids_np).to(cuda_device), cuda_device)
+
+
+def test_noalloc_at_the_size_limit(lib, cuda_device):
+    """A config whose workspace is exactly the scratch array's size: the whole
+    array, its last bytes included, is usable, and the plan matches zb_plan."""
+    cfg = zb.Config(P=8, E=64, K=8, S=515584, H=8, R=1, cap_rows=2 * 515584 * 8)
+    assert zb.workspace_bytes(cfg) == NOALLOC_SCRATCH_BYTES
+    g = torch.Generator(device=cuda_device)
+    g.manual_seed(5)
+    ids = torch.randint(0, cfg.E, (cfg.P, cfg.S, cfg.K), generator=g, device=cuda_device,
+                        dtype=torch.int32)
+    _compare_with_zb_plan(lib, cfg, ids, cuda_device)
+    # one more entry per rank needs more scratch than the array holds
+    over = zb.Config(P=8, E=64, K=8, S=515584 + 256, H=8, R=1)
+    assert zb.workspace_bytes(over) > NOALLOC_SCRATCH_BYTES
+    plan = zb._Plan(*([256] * 10))
+    assert lib.zb_plan_noalloc(ctypes.byref(over.c()), 256, ctypes.byref(plan), None) == \
+        zb.ERR_INVALID
+
+
 def test_noalloc_rejects_configs_beyond_its_scratch(lib, cuda_device):
     big = zb.Config(P=32, E=384, K=16, S=32768, H=8, R=2)
     assert zb.validate(big) == zb.OK

@@ -13,7 +13,11 @@
 //              greedy's max rank load (scores for zb_recalibrate)
 //
 // No kernel waits on another CTA: the chunk prefix each assignment CTA needs
-// is summed directly from the per-chunk histograms.
+// is summed directly from the per-chunk histograms.  The three kernels of a
+// plan are chained by programmatic dependent launch: k_planner and k_assign
+// start while their predecessor finishes, and wait for it (griddepcontrol)
+// only where they read what it writes, so each launch's start-up overlaps the
+// kernel before it.
 //
 // Sources: ISER-MoE "Methodology / HALO-Q Scheduler" (Objectives 1 and 2,
 // stages 1-5); Zepp "4.1 Expert Placement and Token Routing" (R slots per GPU,
@@ -73,6 +77,7 @@ __device__ __forceinline__ int cost_a(int i, int j, int gpn) {
 // Column E of the chunk's row counts ids outside [0, E).
 __global__ void __launch_bounds__(kChunkThreads) k_hist(PlanArgs a) {
   __shared__ int32_t sh[kMaxE + 1];
+  griddep_launch_dependents();  // the planner may launch now and wait for us
   const int c = blockIdx.x, i = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
   const int E = a.E;
   for (int e = tid; e <= E; e += kChunkThreads) sh[e] = 0;
@@ -102,6 +107,14 @@ __global__ void __launch_bounds__(kChunkThreads) k_hist(PlanArgs a) {
   __syncthreads();
   int32_t* out = a.chunk_hist + (int64_t(i) * a.nchunk + c) * (E + 1);
   for (int e = tid; e <= E; e += kChunkThreads) out[e] = sh[e];
+}
+
+// The count row of one source, counts[e] = sum over its chunks of
+// chunk_hist[c][e] (column E: ids outside [0, E)), one thread per column.
+__global__ void __launch_bounds__(kPlanThreads) k_count_row(PlanArgs a, int32_t* counts) {
+  griddep_wait();
+  const int e = blockIdx.x * kPlanThreads + threadIdx.x;
+  if (e <= a.E) counts[e] = strided_sum(a.chunk_hist + e, a.nchunk, a.E + 1);
 }
 
 // ------------------------------------------------------------------ step 2+3
@@ -606,6 +619,10 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
   PlannerSmem s = carve(smem_raw, a);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int P = a.P, E = a.E, R = a.R, Eh = a.Eh, G = Eh + R;
+  // the assignment CTAs may launch now (they read their ids before waiting
+  // for this plan); the chunk histograms are read once k_hist has completed
+  griddep_launch_dependents();
+  griddep_wait();
 
   // route counts cnt[i][e] (and ids outside [0, E)) summed over the chunks
   if (tid == 0) {
@@ -617,13 +634,33 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
   __syncthreads();
   for (int x = tid; x < P * (E + 1); x += kPlanThreads) {
     const int i = x / (E + 1), e = x - i * (E + 1);
-    const int v = strided_sum(a.chunk_hist + int64_t(i) * a.nchunk * (E + 1) + e, a.nchunk,
-                              E + 1);
+    const int v = strided_sum(a.plan_hist + int64_t(i) * a.plan_nchunk * (E + 1) + e,
+                              a.plan_nchunk, E + 1);
     if (e < E) {
       s.cnt[i * E + e] = v;
       a.cnt[i * E + e] = v;
     } else if (v) {
       atomicAdd(&s.misc[kMiscBad], v);
+    }
+  }
+  if (a.own_hist) {
+    // exchanged count rows (one rank of P GPUs): this rank's row must be the
+    // count of its own ids, and every row must be S*K non-negative counts
+    for (int e = tid; e <= E; e += kPlanThreads) {
+      const int own = strided_sum(a.own_hist + e, a.nchunk, E + 1);
+      if (own != a.plan_hist[int64_t(a.src0) * (E + 1) + e]) atomicExch(&s.misc[kMiscErr], 1);
+    }
+    for (int i = warp; i < P; i += kPlanWarps) {
+      long long sum = 0;
+      bool neg = false;
+      for (int e = lane; e <= E; e += 32) {
+        const int v = a.plan_hist[int64_t(i) * (E + 1) + e];
+        neg = neg || v < 0;
+        sum += v;
+      }
+      sum = warp_sum64(sum);
+      if ((__any_sync(kFull, neg) || sum != (long long)a.S * a.K) && lane == 0)
+        atomicExch(&s.misc[kMiscErr], 1);
     }
   }
   // the replica table: empty, or the placement to keep (checked: each slot
@@ -815,19 +852,20 @@ constexpr int kPerWarp = kChunk / kAssignWarps;  // kPerThread steps of 32
 
 // One CTA per (chunk c, source rank i).  Warp w owns entries
 // [kPerWarp*w, kPerWarp*(w+1)) of the chunk and walks them 32 at a time in flat
-// order, so ranks among equal experts come out in flat-index order.
+// order, so ranks among equal experts come out in flat-index order.  The ids
+// and their per-warp histograms depend on nothing the plan writes, so they
+// are done while the planner still runs; the rest waits for it.
 __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
-  if (a.stats[ZB_STAT_STATUS] < 0) return;  // bad ids or capacity: no rows
   __shared__ int32_t wh[kAssignWarps][kMaxE];  // per-warp running position
   __shared__ int32_t s_hoff[kMaxE + 1];
   __shared__ int2 s_seg[kMaxSegWidth];
-  const int c = blockIdx.x, i = blockIdx.y, tid = threadIdx.x, lane = tid & 31,
-            warp = tid >> 5;
+  const int c = blockIdx.x, il = blockIdx.y, i = a.src0 + il, tid = threadIdx.x,
+            lane = tid & 31, warp = tid >> 5;
   const int E = a.E;
   const int64_t nk = int64_t(a.S) * a.K;
   const int64_t start = int64_t(c) * kChunk;
   const int n = (nk - start) < kChunk ? int(nk - start) : kChunk;
-  const int32_t* src = a.ids + int64_t(i) * nk + start;
+  const int32_t* src = a.ids + int64_t(il) * nk + start;
   const int w0 = warp * kPerWarp;
   int ids[kPerThread];
 #pragma unroll
@@ -836,9 +874,6 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
     ids[u] = t < n ? __ldg(src + t) : -1;
   }
   for (int x = tid; x < kAssignWarps * kMaxE; x += kChunkThreads) (&wh[0][0])[x] = 0;
-  for (int e = tid; e <= E; e += kChunkThreads) s_hoff[e] = a.hoff[e];
-  const int2* segrow = a.seg + int64_t(i) * a.seg_width;
-  for (int x = tid; x < a.seg_width; x += kChunkThreads) s_seg[x] = segrow[x];
   __syncthreads();
 
   // pass 1: per-warp histogram of the warp's slice
@@ -848,10 +883,16 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
     const unsigned peers = __match_any_sync(kFull, e);
     if (e >= 0 && lane == __ffs(peers) - 1) wh[warp][e] += __popc(peers);
   }
+
+  griddep_wait();  // the planner has completed: its tables are visible
+  if (a.stats[ZB_STAT_STATUS] < 0) return;  // bad ids or capacity: no rows
+  for (int e = tid; e <= E; e += kChunkThreads) s_hoff[e] = a.hoff[e];
+  const int2* segrow = a.seg + int64_t(i) * a.seg_width;
+  for (int x = tid; x < a.seg_width; x += kChunkThreads) s_seg[x] = segrow[x];
   __syncthreads();
   // exclusive prefix: earlier chunks of this source, then earlier warps
   for (int e = tid; e < E; e += kChunkThreads) {
-    int run = strided_sum(a.chunk_hist + int64_t(i) * a.nchunk * (E + 1) + e, c, E + 1);
+    int run = strided_sum(a.chunk_hist + int64_t(il) * a.nchunk * (E + 1) + e, c, E + 1);
 #pragma unroll
     for (int w = 0; w < kAssignWarps; ++w) {
       const int v = wh[w][e];
@@ -882,9 +923,10 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
         }
         prev = sg.x;
       }
-      const int64_t g = int64_t(i) * nk + start + w0 + 32 * u + lane;
-      a.dst_row[g] = row;
-      if (a.row_src && row >= 0 && int64_t(row) < nrows) a.row_src[row] = int32_t(g);
+      const int64_t f = start + w0 + 32 * u + lane;
+      a.dst_row[int64_t(il) * nk + f] = row;
+      if (a.row_src && row >= 0 && int64_t(row) < nrows)
+        a.row_src[row] = int32_t(int64_t(i) * nk + f);
     }
   }
 }
@@ -982,10 +1024,15 @@ size_t planner_smem_bytes(const zb_config& c) {
   return bytes;
 }
 
-cudaError_t launch_hist(const PlanArgs& a, cudaStream_t s) {
-  if (a.nchunk == 0) return cudaSuccess;
-  k_hist<<<dim3(a.nchunk, a.P), kChunkThreads, 0, s>>>(a);
+cudaError_t launch_hist(const PlanArgs& a, int nsrc, cudaStream_t s) {
+  if (a.nchunk == 0 || nsrc == 0) return cudaSuccess;
+  k_hist<<<dim3(a.nchunk, nsrc), kChunkThreads, 0, s>>>(a);
   return cudaGetLastError();
+}
+
+cudaError_t launch_count_row(const PlanArgs& a, int32_t* counts, cudaStream_t s) {
+  const int blocks = (a.E + 1 + kPlanThreads - 1) / kPlanThreads;
+  return launch_pdl(k_count_row, dim3(blocks), dim3(kPlanThreads), 0, s, a, counts);
 }
 
 template <int kMode, bool kRepair, bool kBand>
@@ -1001,8 +1048,7 @@ cudaError_t launch_planner_mode(const PlanArgs& a, size_t smem, cudaStream_t s) 
     if (err != cudaSuccess) return err;
     configured[dev].store(true, std::memory_order_release);
   }
-  k_planner<kMode, kRepair, kBand><<<1, kPlanThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(k_planner<kMode, kRepair, kBand>, dim3(1), dim3(kPlanThreads), smem, s, a);
 }
 
 template <bool kRepair, bool kBand>
@@ -1044,10 +1090,9 @@ cudaError_t launch_eval_placements(const EvalArgs& ea, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_assign(const PlanArgs& a, cudaStream_t s) {
-  if (a.nchunk == 0) return cudaSuccess;
-  k_assign<<<dim3(a.nchunk, a.P), kChunkThreads, 0, s>>>(a);
-  return cudaGetLastError();
+cudaError_t launch_assign(const PlanArgs& a, int nsrc, cudaStream_t s) {
+  if (a.nchunk == 0 || nsrc == 0) return cudaSuccess;
+  return launch_pdl(k_assign, dim3(a.nchunk, nsrc), dim3(kChunkThreads), 0, s, a);
 }
 
 }  // namespace zb

@@ -66,23 +66,18 @@ int zb_validate(const zb_config* c) {
 
 size_t zb_workspace_bytes(const zb_config* c) {
   if (zb_validate(c) != ZB_OK) return 0;
-  return zb::workspace_layout(*c).bytes;
+  return zb::workspace_layout(*c, c->P).bytes;
 }
 
 }  // extern "C"
 
 namespace {
 
-int plan_impl(const zb_config* c, const int32_t* ids, const int32_t* placement,
-              const zb_plan_t* plan, void* ws, size_t ws_bytes, void* stream) {
-  if (zb_validate(c) != ZB_OK) return ZB_ERR_INVALID;
-  if (!plan_buffers_ok(*c, plan)) return ZB_ERR_INVALID;
-  const Workspace w = zb::workspace_layout(*c);
-  if (!ws || ws_bytes < w.bytes || (reinterpret_cast<uintptr_t>(ws) & 255u)) return ZB_ERR_INVALID;
-  if (c->S > 0 && !ids) return ZB_ERR_INVALID;
-  cudaStream_t s = as_stream(stream);
+// The kernel arguments of a plan over the sources [src0, src0 + nsrc) whose
+// ids, per-chunk histograms and dst_row are laid out from src0.
+zb::PlanArgs plan_args(const zb_config* c, const zb::Workspace& w, const int32_t* ids,
+                       const int32_t* placement, const zb_plan_t* plan, void* ws) {
   char* base = static_cast<char*>(ws);
-
   zb::PlanArgs a{};
   a.P = c->P; a.E = c->E; a.K = c->K; a.S = c->S; a.R = c->R; a.Eh = c->E / c->P;
   a.gpn = c->gpus_per_node; a.cap = c->cap_rows; a.policy = c->policy;
@@ -92,21 +87,43 @@ int plan_impl(const zb_config* c, const int32_t* ids, const int32_t* placement,
   a.nchunk = w.nchunk; a.seg_width = w.seg_width;
   a.ids = ids;
   a.placement = placement;
-  a.cnt = plan->cnt; a.rep_expert = plan->rep_expert; a.rep_quota = plan->rep_quota;
-  a.home_quota = plan->home_quota; a.load_before = plan->load_before;
-  a.load_after = plan->load_after; a.cu_seqlens = plan->cu_seqlens; a.dst_row = plan->dst_row;
-  a.row_src = plan->row_src; a.stats = plan->stats;
+  if (plan) {
+    a.cnt = plan->cnt; a.rep_expert = plan->rep_expert; a.rep_quota = plan->rep_quota;
+    a.home_quota = plan->home_quota; a.load_before = plan->load_before;
+    a.load_after = plan->load_after; a.cu_seqlens = plan->cu_seqlens;
+    a.dst_row = plan->dst_row; a.row_src = plan->row_src; a.stats = plan->stats;
+  }
   a.chunk_hist = reinterpret_cast<int32_t*>(base + w.off_chunk_hist);
   a.hoff = reinterpret_cast<int32_t*>(base + w.off_hoff);
   a.seg = reinterpret_cast<int2*>(base + w.off_seg);
+  a.src0 = 0;
+  a.plan_hist = a.chunk_hist;
+  a.plan_nchunk = w.nchunk;
+  a.own_hist = nullptr;
+  return a;
+}
+
+bool workspace_ok(const void* ws, size_t ws_bytes, size_t need) {
+  return ws && ws_bytes >= need && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0;
+}
+
+int plan_impl(const zb_config* c, const int32_t* ids, const int32_t* placement,
+              const zb_plan_t* plan, void* ws, size_t ws_bytes, void* stream) {
+  if (zb_validate(c) != ZB_OK) return ZB_ERR_INVALID;
+  if (!plan_buffers_ok(*c, plan)) return ZB_ERR_INVALID;
+  const Workspace w = zb::workspace_layout(*c, c->P);
+  if (!workspace_ok(ws, ws_bytes, w.bytes)) return ZB_ERR_INVALID;
+  if (c->S > 0 && !ids) return ZB_ERR_INVALID;
+  cudaStream_t s = as_stream(stream);
+  const zb::PlanArgs a = plan_args(c, w, ids, placement, plan, ws);
 
   if (a.row_src &&
       cudaMemsetAsync(a.row_src, 0xff, sizeof(int32_t) * size_t(c->P) * c->cap_rows, s) !=
           cudaSuccess)
     return ZB_ERR_CUDA;
-  if (zb::launch_hist(a, s) != cudaSuccess) return ZB_ERR_CUDA;
+  if (zb::launch_hist(a, c->P, s) != cudaSuccess) return ZB_ERR_CUDA;
   if (zb::launch_planner(a, zb::planner_smem_bytes(*c), s) != cudaSuccess) return ZB_ERR_CUDA;
-  if (zb::launch_assign(a, s) != cudaSuccess) return ZB_ERR_CUDA;
+  if (zb::launch_assign(a, c->P, s) != cudaSuccess) return ZB_ERR_CUDA;
   return ZB_OK;
 }
 
@@ -123,6 +140,43 @@ int zb_plan_placed(const zb_config* c, const int32_t* ids, const int32_t* placem
                    const zb_plan_t* plan, void* ws, size_t ws_bytes, void* stream) {
   if (c && c->R > 0 && !placement) return ZB_ERR_INVALID;
   return plan_impl(c, ids, c && c->R > 0 ? placement : nullptr, plan, ws, ws_bytes, stream);
+}
+
+size_t zb_rank_workspace_bytes(const zb_config* c) {
+  if (zb_validate(c) != ZB_OK) return 0;
+  return zb::workspace_layout(*c, 1).bytes;
+}
+
+int zb_count(const zb_config* c, const int32_t* ids, int32_t* counts, void* ws,
+             size_t ws_bytes, void* stream) {
+  if (zb_validate(c) != ZB_OK || !counts) return ZB_ERR_INVALID;
+  const Workspace w = zb::workspace_layout(*c, 1);
+  if (!workspace_ok(ws, ws_bytes, w.bytes)) return ZB_ERR_INVALID;
+  if (c->S > 0 && !ids) return ZB_ERR_INVALID;
+  cudaStream_t s = as_stream(stream);
+  const zb::PlanArgs a = plan_args(c, w, ids, nullptr, nullptr, ws);
+  if (zb::launch_hist(a, 1, s) != cudaSuccess) return ZB_ERR_CUDA;
+  if (zb::launch_count_row(a, counts, s) != cudaSuccess) return ZB_ERR_CUDA;
+  return ZB_OK;
+}
+
+int zb_plan_rank(const zb_config* c, int rank, const int32_t* counts, const int32_t* ids,
+                 const int32_t* placement, const zb_plan_t* plan, void* ws, size_t ws_bytes,
+                 void* stream) {
+  if (zb_validate(c) != ZB_OK || rank < 0 || rank >= c->P || !counts) return ZB_ERR_INVALID;
+  if (!plan_buffers_ok(*c, plan) || plan->row_src) return ZB_ERR_INVALID;
+  const Workspace w = zb::workspace_layout(*c, 1);
+  if (!workspace_ok(ws, ws_bytes, w.bytes)) return ZB_ERR_INVALID;
+  if (c->S > 0 && !ids) return ZB_ERR_INVALID;
+  cudaStream_t s = as_stream(stream);
+  zb::PlanArgs a = plan_args(c, w, ids, c->R > 0 ? placement : nullptr, plan, ws);
+  a.src0 = rank;
+  a.plan_hist = counts;
+  a.plan_nchunk = 1;
+  a.own_hist = a.chunk_hist;
+  if (zb::launch_planner(a, zb::planner_smem_bytes(*c), s) != cudaSuccess) return ZB_ERR_CUDA;
+  if (zb::launch_assign(a, 1, s) != cudaSuccess) return ZB_ERR_CUDA;
+  return ZB_OK;
 }
 
 int zb_plan_status(const zb_config* c, const zb_plan_t* plan, void* stream, int32_t* max_load) {
@@ -207,6 +261,40 @@ int zb_combine_merged(const zb_config* c, const zb_plan_t* plan, const zb_merge_
   if ((part && !aligned16(part)) || (out && !aligned16(out))) return ZB_ERR_INVALID;
   if (zb::launch_combine_merged(c->P, c->S, c->K, c->H, c->cap_rows, m->tok_row, plan->stats,
                                 part, out, as_stream(stream)) != cudaSuccess)
+    return ZB_ERR_CUDA;
+  return ZB_OK;
+}
+
+int zb_dispatch_rank(const zb_config* c, const zb_plan_t* plan, const uint16_t* hidden,
+                     uint16_t* const* bufs, void* stream) {
+  if (zb_validate(c) != ZB_OK || !plan || !plan->stats || !bufs) return ZB_ERR_INVALID;
+  if (c->S > 0 && (!plan->dst_row || !hidden)) return ZB_ERR_INVALID;
+  if (hidden && !aligned16(hidden)) return ZB_ERR_INVALID;
+  zb::RankBufs t{};
+  for (int j = 0; j < c->P; ++j) {
+    if (!bufs[j] || !aligned16(bufs[j])) return ZB_ERR_INVALID;
+    t.p[j] = bufs[j];
+  }
+  if (zb::launch_dispatch_ranks(c->P, c->S, c->K, c->H, c->cap_rows, plan->dst_row, plan->stats,
+                                hidden, t, as_stream(stream)) != cudaSuccess)
+    return ZB_ERR_CUDA;
+  return ZB_OK;
+}
+
+int zb_combine_rank(const zb_config* c, const zb_plan_t* plan, const uint16_t* const* ys,
+                    const float* w, uint16_t* out, void* stream) {
+  if (zb_validate(c) != ZB_OK || !plan || !plan->stats || !ys) return ZB_ERR_INVALID;
+  if (c->S > 0 && (!plan->dst_row || !w || !out)) return ZB_ERR_INVALID;
+  if (out && !aligned16(out)) return ZB_ERR_INVALID;
+  zb::RankBufs t{};
+  bool wide_ok = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
+  for (int j = 0; j < c->P; ++j) {
+    if (!ys[j] || !aligned16(ys[j])) return ZB_ERR_INVALID;
+    t.p[j] = const_cast<uint16_t*>(ys[j]);
+    wide_ok = wide_ok && (reinterpret_cast<uintptr_t>(ys[j]) & 31u) == 0;
+  }
+  if (zb::launch_combine_ranks(c->P, c->S, c->K, c->H, c->cap_rows, plan->dst_row, plan->stats,
+                               t, w, out, wide_ok, as_stream(stream)) != cudaSuccess)
     return ZB_ERR_CUDA;
   return ZB_OK;
 }

@@ -4,6 +4,8 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <utility>
+
 #include <cuda_runtime.h>
 
 #include "zb.h"
@@ -27,7 +29,9 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Layout of the scratch workspace (all offsets 256-byte aligned).  Nothing in
 // it needs initialising: every word is written before it is read.
-//   chunk_hist int32 [P][nchunk][E+1]  per-chunk expert counts; column E
+//   chunk_hist int32 [nsrc][nchunk][E+1]  per-chunk expert counts of the
+//                                      sources histogrammed here (all P on one
+//                                      GPU, or one rank's own); column E
 //                                      counts the chunk's ids outside [0, E)
 //   hoff       int32 [E+1]             first segment of expert e in a row of seg
 //   seg        int2  [P][E + P*R]      per (source i, expert e): the hosts in
@@ -39,14 +43,14 @@ struct Workspace {
   size_t off_chunk_hist, off_hoff, off_seg, bytes;
 };
 
-inline Workspace workspace_layout(const zb_config& c) {
+inline Workspace workspace_layout(const zb_config& c, int nsrc) {
   Workspace w{};
   const int64_t nk = int64_t(c.S) * c.K;
   w.nchunk = int(ceil_div(nk, kChunk));
   w.seg_width = c.E + c.P * c.R;
   size_t o = 0;
   w.off_chunk_hist = o;
-  o = align256(o + sizeof(int32_t) * size_t(c.P) * w.nchunk * (c.E + 1));
+  o = align256(o + sizeof(int32_t) * size_t(nsrc) * w.nchunk * (c.E + 1));
   w.off_hoff = o;
   o = align256(o + sizeof(int32_t) * size_t(c.E + 1));
   w.off_seg = o;
@@ -56,11 +60,24 @@ inline Workspace workspace_layout(const zb_config& c) {
 }
 
 // Kernel parameter block shared by the plan kernels.
+//
+// The planner reads the route counts from plan_hist [P][plan_nchunk][E+1],
+// summing each column over its chunks: the per-chunk histograms of every
+// source (whole batch on one GPU), or the exchanged count rows of P ranks
+// (plan_nchunk = 1).  k_hist and k_assign handle the sources src0 ..
+// src0 + gridDim.y - 1; ids, dst_row and chunk_hist are indexed from src0
+// (local), seg and row_src by the global source.  own_hist, when set, holds
+// the per-chunk histograms of source src0 alone, which the planner checks
+// against its row of plan_hist.
 struct PlanArgs {
   int P, E, K, S, R, Eh, gpn, cap, policy;
   int relax, cfix;  // eq. (1)'s band: C as floor(C * 2^20), 0 unless relax
   int repair;       // quota repair between rank pairs after the greedy
   int nchunk, seg_width;
+  int src0;
+  int plan_nchunk;
+  const int32_t* plan_hist;
+  const int32_t* own_hist;
   const int32_t* ids;
   const int32_t* placement;  // [P][R] replica placement to keep, or nullptr
   int32_t* cnt;
@@ -105,17 +122,59 @@ struct MergeArgs {
   int32_t* chunk_cnt;  // workspace [nchunk][P]
 };
 
+// Programmatic dependent launch.  A kernel launched with launch_pdl may start
+// while the kernel before it on the stream is still running, once every CTA
+// of that kernel has called griddep_launch_dependents (or exited).  Before
+// it touches anything its predecessor writes, it calls griddep_wait, which
+// returns once the predecessor has completed and its writes are visible.
+// Without a pending dependency (a plain launch) griddep_wait returns at once.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 size_t planner_smem_bytes(const zb_config& c);
 
-cudaError_t launch_hist(const PlanArgs& a, cudaStream_t s);
+cudaError_t launch_hist(const PlanArgs& a, int nsrc, cudaStream_t s);
+cudaError_t launch_count_row(const PlanArgs& a, int32_t* counts, cudaStream_t s);
 cudaError_t launch_planner(const PlanArgs& a, size_t smem, cudaStream_t s);
-cudaError_t launch_assign(const PlanArgs& a, cudaStream_t s);
+cudaError_t launch_assign(const PlanArgs& a, int nsrc, cudaStream_t s);
 size_t eval_smem_bytes(int P, int E, int R);
 cudaError_t launch_eval_placements(const EvalArgs& ea, cudaStream_t s);
+
+// Receive buffers of the P ranks: one per rank (base pointers; for one
+// buffer holding every rank's rows, rank j's base is buf + j*cap*H).
+struct RankBufs {
+  uint16_t* p[kMaxP];
+};
 
 cudaError_t launch_dispatch(int P, int S, int K, int H, int cap, const int32_t* dst_row,
                             const int64_t* stats, const uint16_t* hidden, uint16_t* buf,
                             cudaStream_t s);
+cudaError_t launch_dispatch_ranks(int P, int ntok, int K, int H, int cap,
+                                  const int32_t* dst_row, const int64_t* stats,
+                                  const uint16_t* hidden, const RankBufs& bufs, cudaStream_t s);
+cudaError_t launch_combine_ranks(int P, int ntok, int K, int H, int cap, const int32_t* dst_row,
+                                 const int64_t* stats, const RankBufs& ys, const float* w,
+                                 uint16_t* out, bool wide_ok, cudaStream_t s);
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t s);
 cudaError_t launch_dispatch_merged(int P, int S, int K, int H, int cap, const int32_t* tok_row,
                                    const int64_t* stats, const uint16_t* hidden, uint16_t* tbuf,

@@ -26,7 +26,9 @@ std::mutex g_lock;
 void* g_addr[kMaxDevices] = {};
 
 // Device address of the scratch array on the calling thread's current device,
-// looked up once per device (with that device current) and cached.
+// looked up once per device (with that device current) and cached for the life
+// of the process.  A device reset reloads the module, so the header tells
+// callers not to use this entry point on a device after resetting it.
 int scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ZB_ERR_CUDA;

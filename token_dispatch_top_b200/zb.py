@@ -37,7 +37,9 @@ STATS_LEN = 8
 EXPORTS = ("zb_strerror", "zb_validate", "zb_workspace_bytes", "zb_plan", "zb_plan_placed",
            "zb_plan_status", "zb_dispatch", "zb_combine", "zb_merge_workspace_bytes",
            "zb_merge", "zb_dispatch_merged", "zb_combine_reduce", "zb_combine_merged",
-           "zb_recalibrate_workspace_bytes", "zb_recalibrate", "zb_place_by_demand")
+           "zb_recalibrate_workspace_bytes", "zb_recalibrate", "zb_place_by_demand",
+           "zb_rank_workspace_bytes", "zb_count", "zb_plan_rank", "zb_dispatch_rank",
+           "zb_combine_rank")
 
 
 class ZbError(RuntimeError):
@@ -99,6 +101,13 @@ def load() -> ctypes.CDLL:
         lib.zb_recalibrate.argtypes = [cfgp, vp, vp, ctypes.c_int, ctypes.c_float, ctypes.c_int,
                                        vp, ctypes.c_size_t, vp, i32p, i32p]
         lib.zb_place_by_demand.argtypes = [cfgp, vp, vp]
+        lib.zb_rank_workspace_bytes.argtypes = [cfgp]
+        lib.zb_rank_workspace_bytes.restype = ctypes.c_size_t
+        lib.zb_count.argtypes = [cfgp, vp, vp, vp, ctypes.c_size_t, vp]
+        lib.zb_plan_rank.argtypes = [cfgp, ctypes.c_int, vp, vp, vp, planp, vp, ctypes.c_size_t,
+                                     vp]
+        lib.zb_dispatch_rank.argtypes = [cfgp, planp, vp, ctypes.POINTER(ctypes.c_void_p), vp]
+        lib.zb_combine_rank.argtypes = [cfgp, planp, ctypes.POINTER(ctypes.c_void_p), vp, vp, vp]
         _lib = lib
     return _lib
 
@@ -359,3 +368,128 @@ def place_by_demand(cfg: Config, demand) -> np.ndarray:
     if st != OK:
         raise ZbError(st, "zb_place_by_demand")
     return pl
+
+
+# --------------------------------------------------- the path on one of P GPUs
+
+class RankPlan:
+    """Device buffers of the plan of one rank of P GPUs: the plan tables (as
+    :class:`Plan`), ``dst_row`` [S,K] for this rank's entries, this rank's
+    count row ``counts`` [E+1], the all-gathered table ``table`` [P,E+1] and
+    the scratch workspace that ``count`` fills and ``plan_rank`` reads."""
+
+    def __init__(self, cfg: Config, rank: int, device):
+        if validate(cfg) != OK or not 0 <= rank < cfg.P:
+            raise ZbError(ERR_INVALID, f"config {cfg}, rank {rank}")
+        i32 = dict(dtype=torch.int32, device=device)
+        P, E, R = cfg.P, cfg.E, cfg.R
+        self.cfg, self.rank = cfg, rank
+        self.cnt = torch.empty((P, E), **i32)
+        self.rep_expert = torch.empty((P, R), **i32)
+        self.rep_quota = torch.empty((P, R), **i32)
+        self.home_quota = torch.empty((E,), **i32)
+        self.load_before = torch.empty((P,), **i32)
+        self.load_after = torch.empty((P,), **i32)
+        self.cu_seqlens = torch.empty((P, cfg.Eh + R + 1), **i32)
+        self.dst_row = torch.empty((cfg.S, cfg.K), **i32)
+        self.stats = torch.zeros((STATS_LEN,), dtype=torch.int64, device=device)
+        self.counts = torch.empty((E + 1,), **i32)
+        self.table = torch.empty((P, E + 1), **i32)
+        self.ws_bytes = int(load().zb_rank_workspace_bytes(ctypes.byref(cfg.c())))
+        self.workspace = torch.empty((self.ws_bytes + 256,), dtype=torch.uint8, device=device)
+        self.ws_ptr = (self.workspace.data_ptr() + 255) & ~255
+        self._c = cfg.c()
+
+        def p(t):
+            return None if t is None or t.numel() == 0 else t.data_ptr()
+        self._p = _Plan(p(self.cnt), p(self.rep_expert), p(self.rep_quota), p(self.home_quota),
+                        p(self.load_before), p(self.load_after), p(self.cu_seqlens),
+                        p(self.dst_row), None, p(self.stats))
+
+
+def count(rp: RankPlan, topk_ids: torch.Tensor, stream=None) -> None:
+    """Step 1 on one rank (asynchronous): ``rp.counts`` = the per-expert counts
+    of this rank's ids int32 [S,K], then the number of ids outside [0, E)."""
+    cfg = rp.cfg
+    _check(topk_ids, (cfg.S, cfg.K), torch.int32, "topk_ids")
+    st = load().zb_count(ctypes.byref(rp._c), topk_ids.data_ptr(), rp.counts.data_ptr(),
+                         rp.ws_ptr, rp.ws_bytes, _stream(stream))
+    if st != OK:
+        raise ZbError(st, "zb_count")
+
+
+def exchange_counts(counts: torch.Tensor, table: torch.Tensor, group=None) -> torch.Tensor:
+    """The count exchange: every rank's ``counts`` row [E+1] gathered, in rank
+    order, into ``table`` [P,E+1] with torch.distributed (NCCL on GPUs; any
+    backend whose all-gather takes these tensors).  Without an initialised
+    process group, P must be 1."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        if table.shape[0] != 1:
+            raise ZbError(ERR_INVALID, "exchange_counts: no process group and P > 1")
+        table[0].copy_(counts)
+        return table
+    if dist.get_world_size(group) != table.shape[0]:
+        raise ZbError(ERR_INVALID, "exchange_counts: world size differs from P")
+    dist.all_gather(list(table.unbind(0)), counts, group=group)
+    return table
+
+
+def plan_rank(rp: RankPlan, topk_ids: torch.Tensor, placement: torch.Tensor | None = None,
+              stream=None) -> None:
+    """Steps 2-3 on one rank (asynchronous), from ``rp.table`` (the exchanged
+    counts) and this rank's ids; ``count`` must have run on the same ids."""
+    cfg = rp.cfg
+    _check(topk_ids, (cfg.S, cfg.K), torch.int32, "topk_ids")
+    _check(rp.table, (cfg.P, cfg.E + 1), torch.int32, "table")
+    pl = None
+    if placement is not None:
+        _check(placement, (cfg.P, cfg.R), torch.int32, "placement")
+        pl = placement.data_ptr() if placement.numel() else None
+    st = load().zb_plan_rank(ctypes.byref(rp._c), rp.rank, rp.table.data_ptr(),
+                             topk_ids.data_ptr(), pl, ctypes.byref(rp._p), rp.ws_ptr,
+                             rp.ws_bytes, _stream(stream))
+    if st != OK:
+        raise ZbError(st, "zb_plan_rank")
+
+
+def _pointer_table(cfg: Config, rows, what: str):
+    """A host array of P device pointers from P tensors bf16 [cap,H] or P
+    integer addresses (peer memory mapped into this process)."""
+    if len(rows) != cfg.P:
+        raise ZbError(ERR_INVALID, f"{what}: want {cfg.P} buffers, got {len(rows)}")
+    tbl = (ctypes.c_void_p * cfg.P)()
+    for j, r in enumerate(rows):
+        if isinstance(r, torch.Tensor):
+            _check(r, (cfg.cap, cfg.H), torch.bfloat16, f"{what}[{j}]")
+            tbl[j] = r.data_ptr()
+        else:
+            tbl[j] = int(r)
+    return tbl
+
+
+def dispatch_rank(rp: RankPlan, hidden: torch.Tensor, bufs, stream=None) -> None:
+    """Step 4 on one rank (asynchronous): ``hidden`` bf16 [S,H] into the P
+    receive buffers ``bufs`` (bf16 [cap,H] tensors or device addresses)."""
+    cfg = rp.cfg
+    _check(hidden, (cfg.S, cfg.H), torch.bfloat16, "hidden")
+    tbl = _pointer_table(cfg, bufs, "bufs")
+    st = load().zb_dispatch_rank(ctypes.byref(rp._c), ctypes.byref(rp._p), hidden.data_ptr(),
+                                 tbl, _stream(stream))
+    if st != OK:
+        raise ZbError(st, "zb_dispatch_rank")
+
+
+def combine_rank(rp: RankPlan, ys, topk_weights: torch.Tensor, out: torch.Tensor,
+                 stream=None) -> None:
+    """Step 5 on one rank (asynchronous): this rank's tokens gathered from the
+    P expert-output buffers ``ys`` (bf16 [cap,H] tensors or device addresses)
+    with ``topk_weights`` fp32 [S,K] into ``out`` bf16 [S,H]."""
+    cfg = rp.cfg
+    _check(topk_weights, (cfg.S, cfg.K), torch.float32, "topk_weights")
+    _check(out, (cfg.S, cfg.H), torch.bfloat16, "out")
+    tbl = _pointer_table(cfg, ys, "ys")
+    st = load().zb_combine_rank(ctypes.byref(rp._c), ctypes.byref(rp._p), tbl,
+                                topk_weights.data_ptr(), out.data_ptr(), _stream(stream))
+    if st != OK:
+        raise ZbError(st, "zb_combine_rank")
