@@ -173,6 +173,13 @@ def test_random_shapes_every_option(dev, k):
                     _rand_bits(rng, (zc.P * zc.cap, zc.H)), w, dev, separate=bool(k % 3 == 0))
 
 
+def _device_status(rp) -> int:
+    """The plan's status as the planner recorded it (the binding's plan_status
+    raises on ERR_INVALID, which is also its code for a bad argument)."""
+    torch.cuda.synchronize()
+    return int(rp.stats[zb.STAT_STATUS])
+
+
 def test_inconsistent_counts_and_bad_ids(dev):
     rng = np.random.default_rng(11)
     zc = zb.Config(P=4, E=8, K=2, S=50, H=16, R=1, cap_rows=400)
@@ -186,7 +193,7 @@ def test_inconsistent_counts_and_bad_ids(dev):
     if not torch.equal(t[1], torch.from_numpy(table[1]).to(dev)):
         rp.table.copy_(t)
         zb.plan_rank(rp, torch.from_numpy(ids[1]).to(dev))
-        assert zb.plan_status(rp)[0] == zb.ERR_INVALID
+        assert _device_status(rp) == zb.ERR_INVALID
         hid = torch.randn((50, 16), device=dev).to(torch.bfloat16)
         bufs = [torch.full((400, 16), parity.SENTINEL, dtype=torch.int16, device=dev)
                 .view(torch.bfloat16) for _ in range(4)]
@@ -198,7 +205,7 @@ def test_inconsistent_counts_and_bad_ids(dev):
     t[3, 0] += 1
     rps[0].table.copy_(t)
     zb.plan_rank(rps[0], torch.from_numpy(ids[0]).to(dev))
-    assert zb.plan_status(rps[0])[0] == zb.ERR_INVALID
+    assert _device_status(rps[0]) == zb.ERR_INVALID
     # an id out of range on rank 2 fails every rank alike
     ids2 = ids.copy()
     ids2[2, 7, 1] = -5

@@ -50,23 +50,64 @@ __device__ __forceinline__ long long warp_sum64(long long v) {
   return v;
 }
 
-// Sum of col[0], col[stride], ..., col[(n-1)*stride], eight loads in flight.
+// Sum of col[0], col[stride], ..., col[(n-1)*stride], kInFlight loads in
+// flight.
+template <int kInFlight = 8>
 __device__ __forceinline__ int strided_sum(const int32_t* col, int n, int64_t stride) {
   int v = 0;
-  for (int c = 0; c < n; c += 8) {
-    int x[8];
+  for (int c = 0; c < n; c += kInFlight) {
+    int x[kInFlight];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) x[u] = c + u < n ? col[int64_t(c + u) * stride] : 0;
+    for (int u = 0; u < kInFlight; ++u) x[u] = c + u < n ? col[int64_t(c + u) * stride] : 0;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) v += x[u];
+    for (int u = 0; u < kInFlight; ++u) v += x[u];
   }
   return v;
 }
 
+// Column sums of a [rows][nchunk][ncol_row] table for the four columns
+// x0 + u*step (u < 4) of the flattened [rows][ncol_row] index space below
+// ncol: v[u] = sum over c of table[row][c][col].  Thirty-two loads in flight
+// per thread.
+__device__ __forceinline__ void column_sums4(const int32_t* table, int nchunk, int ncol_row,
+                                             int ncol, int x0, int step, int (&v)[4]) {
+  const int32_t* col[4];
+  bool ok[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int x = x0 + u * step;
+    ok[u] = x < ncol;
+    const int i = ok[u] ? x / ncol_row : 0, e = ok[u] ? x - i * ncol_row : 0;
+    col[u] = table + int64_t(i) * nchunk * ncol_row + e;
+    v[u] = 0;
+  }
+  for (int c = 0; c < nchunk; c += 8) {
+    int t[4][8];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        t[u][k] = (ok[u] && c + k < nchunk) ? col[u][int64_t(c + k) * ncol_row] : 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[u] += t[u][k];
+  }
+}
+
+// r / g for the planner's small non-negative integers (ranks, experts), from
+// inv = float(1/g): (r + 1/2) / g lies at least 1/(2g) from an integer, and
+// for r < 2^22 the float product (r + 1/2) * inv is within (r + 1/2) / g *
+// 2^-23 < 1/(2g) of it, so truncating it gives r / g exactly.  Two float
+// instructions instead of an integer division by a runtime value.
+__device__ __forceinline__ int div_small(int r, float inv) {
+  return int((float(r) + 0.5f) * inv);
+}
+
 // a_ij of eq. (1): 0 same rank; 1 other rank (flat) or same node; 4 other node.
-__device__ __forceinline__ int cost_a(int i, int j, int gpn) {
+__device__ __forceinline__ int cost_a(int i, int j, int gpn, float inv_gpn) {
   if (i == j) return 0;
-  if (gpn > 1 && (i / gpn) != (j / gpn)) return 4;
+  if (gpn > 1 && div_small(i, inv_gpn) != div_small(j, inv_gpn)) return 4;
   return 1;
 }
 
@@ -114,7 +155,7 @@ __global__ void __launch_bounds__(kChunkThreads) k_hist(PlanArgs a) {
 __global__ void __launch_bounds__(kPlanThreads) k_count_row(PlanArgs a, int32_t* counts) {
   griddep_wait();
   const int e = blockIdx.x * kPlanThreads + threadIdx.x;
-  if (e <= a.E) counts[e] = strided_sum(a.chunk_hist + e, a.nchunk, a.E + 1);
+  if (e <= a.E) counts[e] = strided_sum<16>(a.chunk_hist + e, a.nchunk, a.E + 1);
 }
 
 // ------------------------------------------------------------------ step 2+3
@@ -155,8 +196,9 @@ __device__ PlannerSmem carve(char* base, const PlanArgs& a) {
 
 enum {
   kMiscT = 0, kMiscMax = 1, kMiscNrep = 2, kMiscIters = 3, kMiscBad = 4, kMiscErr = 5,
-  kMiscRecv = 6,     // banded plans: the most rows any rank receives
-  kMiscRepaired = 7  // rows moved by quota repair, per direction
+  kMiscRecv = 6,      // banded plans: the most rows any rank receives
+  kMiscRepaired = 7,  // rows moved by quota repair, per direction
+  kMiscNRepExp = 8    // experts with at least one replica (first in order)
 };
 
 // Greedy replica placement, run by one warp; lane r holds rank r's load,
@@ -173,6 +215,7 @@ __device__ void greedy_warp(const PlanArgs& a, PlannerSmem& s, int T, int load, 
   // mask of the ranks on lane's node
   const unsigned node_mask =
       gpn >= 32 ? kFull : (((1u << gpn) - 1u) << ((lane / gpn) * gpn));
+  const int my_node = lane / gpn;
   for (int guard = 0; guard <= max_iters; ++guard) {
     // donor: the busiest non-stuck rank, ties to the lowest rank
     const unsigned dl = stuck ? 0u : unsigned(load) + 1u;
@@ -186,13 +229,15 @@ __device__ void greedy_warp(const PlanArgs& a, PlannerSmem& s, int T, int load, 
     const unsigned base = __ballot_sync(kFull, lane < P && lane != d && nfill < R && load < T);
     // d's heaviest home expert (largest remaining quota, ties: lowest id)
     // that some rank in base can take (it holds no copy yet)
-    unsigned bq = 0u, bx = 0xffffffffu;
+    unsigned bq = 0u, bx = 0xffffffffu, bh = 0u;
     for (int x = lane; x < Eh; x += 32) {
       const int e = d * Eh + x;
       const unsigned q = unsigned(s.hq[e]);
-      if (q > 0u && (base & ~s.hold[e]) != 0u && q > bq) {
+      const unsigned h = s.hold[e];
+      if (q > 0u && (base & ~h) != 0u && q > bq) {
         bq = q;
         bx = unsigned(x);
+        bh = h;
       }
     }
     const unsigned qmax = __reduce_max_sync(kFull, bq);
@@ -203,11 +248,12 @@ __device__ void greedy_warp(const PlanArgs& a, PlannerSmem& s, int T, int load, 
     const unsigned xmin = __reduce_min_sync(kFull, bq == qmax ? bx : 0xffffffffu);
     const int e = d * Eh + int(xmin);
     const int q = int(qmax);
-    const unsigned hold = s.hold[e];
+    // the holders of e, from the lane that examined it (x = xmin there)
+    const unsigned hold = __shfl_sync(kFull, bh, int(xmin & 31u));
     // receiver: a node without the expert first, then the lowest load, then
-    // the lowest rank
+    // the lowest rank (e is homed on the donor d)
     const bool elig = ((base >> lane) & 1u) && !((hold >> lane) & 1u);
-    const bool cov = ((e / Eh) / gpn == lane / gpn) || ((hold & node_mask) != 0u);
+    const bool cov = (__shfl_sync(kFull, my_node, d) == my_node) || ((hold & node_mask) != 0u);
     int r, rload;
     if (kPolicy == ZB_POLICY_LOCAL) {
       // balance first, locality among equal moves (HALO-Q Objective 2): after
@@ -442,7 +488,7 @@ __device__ void flows_exact(const PlanArgs& a, PlannerSmem& s, int e, int h0,
       const int j = __ffs(hm) - 1;
       hm &= hm - 1u;
       const int rem = qw[t];
-      const int v = (lane < P && cost_a(lane, j, gpn) == lev) ? dres : 0;
+      const int v = (lane < P && cost_a(lane, j, gpn, a.inv_gpn) == lev) ? dres : 0;
       const int inc = warp_incl_scan(v, lane);
       const int take = max(0, min(v, rem - (inc - v)));
       const int tot = int(__reduce_add_sync(kFull, unsigned(take)));
@@ -501,7 +547,7 @@ __device__ int flows_band(const PlanArgs& a, PlannerSmem& s, int e, int h0, unsi
       const int hij = __shfl_sync(kFull, hi, j);
       const int need = max(loj - rj, 0);
       const int avail = need + min(hij - max(rj, loj), slack);
-      const int v = (lane < P && cost_a(lane, j, gpn) == lev) ? dres : 0;
+      const int v = (lane < P && cost_a(lane, j, gpn, a.inv_gpn) == lev) ? dres : 0;
       const int inc = warp_incl_scan(v, lane);
       const int take = max(0, min(v, avail - (inc - v)));
       const int tot = int(__reduce_add_sync(kFull, unsigned(take)));
@@ -532,7 +578,7 @@ __device__ long long emit_segments(const PlanArgs& a, const PlannerSmem& s, int 
       const int j = __ffs(hm) - 1;
       hm &= hm - 1u;
       const int m = Mw[t * 32 + lane];
-      cost += (long long)cost_a(lane, j, gpn) * m;
+      cost += (long long)cost_a(lane, j, gpn, a.inv_gpn) * m;
       const int inc = warp_incl_scan(m, lane);
       __syncwarp();
       Mw[t * 32 + lane] = inc;  // inclusive prefix over sources
@@ -547,7 +593,7 @@ __device__ long long emit_segments(const PlanArgs& a, const PlannerSmem& s, int 
       for (int t = 0; t < nh; ++t) {
         const int j = __ffs(hm) - 1;
         hm &= hm - 1u;
-        if (cost_a(lane, j, gpn) != want) continue;
+        if (cost_a(lane, j, gpn, a.inv_gpn) != want) continue;
         const int inc = Mw[t * 32 + lane];
         const int prev = lane > 0 ? Mw[t * 32 + lane - 1] : 0;
         int grp;
@@ -576,7 +622,7 @@ template <bool kBand, bool kEmit>
 __device__ long long transport_warp(const PlanArgs& a, PlannerSmem& s, int e, int lane,
                                     int32_t* Mw, int32_t* qw) {
   const int P = a.P, Eh = a.Eh, G = Eh + a.R, gpn = a.gpn;
-  const int h0 = e / Eh;
+  const int h0 = div_small(e, a.inv_eh);
   const unsigned hold = s.hold[e];
   const int d = lane < P ? s.cnt[lane * a.E + e] : 0;
   int2* seg = a.seg + int64_t(lane) * a.seg_width + s.hoff[e];
@@ -589,7 +635,7 @@ __device__ long long transport_warp(const PlanArgs& a, PlannerSmem& s, int e, in
     const int inc = warp_incl_scan(d, lane);
     if (lane < P)
       seg[0] = make_int2(d, h0 * a.cap + s.cu[h0 * (G + 1) + (e - h0 * Eh)] + inc - d);
-    return (long long)cost_a(lane, h0, gpn) * d;
+    return (long long)cost_a(lane, h0, gpn, a.inv_gpn) * d;
   }
   const unsigned hostmask = hold | (1u << h0);
   const int nh = __popc(hostmask);
@@ -632,22 +678,28 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
     s_cost = 0ull;
   }
   __syncthreads();
-  for (int x = tid; x < P * (E + 1); x += kPlanThreads) {
-    const int i = x / (E + 1), e = x - i * (E + 1);
-    const int v = strided_sum(a.plan_hist + int64_t(i) * a.plan_nchunk * (E + 1) + e,
-                              a.plan_nchunk, E + 1);
-    if (e < E) {
-      s.cnt[i * E + e] = v;
-      a.cnt[i * E + e] = v;
-    } else if (v) {
-      atomicAdd(&s.misc[kMiscBad], v);
+  // (four columns per thread at a time, eight chunks of each in flight)
+  for (int x0 = tid; x0 < P * (E + 1); x0 += 4 * kPlanThreads) {
+    int v[4];
+    column_sums4(a.plan_hist, a.plan_nchunk, E + 1, P * (E + 1), x0, kPlanThreads, v);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int x = x0 + u * kPlanThreads;
+      if (x >= P * (E + 1)) break;
+      const int i = x / (E + 1), e = x - i * (E + 1);
+      if (e < E) {
+        s.cnt[i * E + e] = v[u];
+        a.cnt[i * E + e] = v[u];
+      } else if (v[u]) {
+        atomicAdd(&s.misc[kMiscBad], v[u]);
+      }
     }
   }
   if (a.own_hist) {
     // exchanged count rows (one rank of P GPUs): this rank's row must be the
     // count of its own ids, and every row must be S*K non-negative counts
     for (int e = tid; e <= E; e += kPlanThreads) {
-      const int own = strided_sum(a.own_hist + e, a.nchunk, E + 1);
+      const int own = strided_sum<16>(a.own_hist + e, a.nchunk, E + 1);
       if (own != a.plan_hist[int64_t(a.src0) * (E + 1) + e]) atomicExch(&s.misc[kMiscErr], 1);
     }
     for (int i = warp; i < P; i += kPlanWarps) {
@@ -774,6 +826,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
         if (take) s.order[n + __popc(m & ((1u << lane) - 1u))] = e;
         n += __popc(m);
       }
+      if (pass == 0 && lane == 0) s.misc[kMiscNRepExp] = n;
     }
   }
   int32_t* Mw = s.M + warp * 32 * 32;
@@ -820,9 +873,29 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
   const int rows_max = kBand ? s.misc[kMiscRecv] : max_load;
   const bool capacity = rows_max > a.cap;
   long long cost_part = 0;
-  if (!capacity)
-    for (int k = warp; k < E; k += kPlanWarps)
+  if (!capacity) {
+    // experts with replicas: the transport of eq. (1), one warp each
+    const int nrx = s.misc[kMiscNRepExp];
+    for (int k = warp; k < nrx; k += kPlanWarps)
       cost_part += transport_warp<kBand, true>(a, s, s.order[k], lane, Mw, qw);
+    // experts served by their home rank alone: every source sends it all its
+    // rows, one segment per source; a thread per expert walks the sources
+    // in rank order (the same segments transport_warp's home-only case
+    // writes, without a warp scan per expert)
+    for (int k = nrx + tid; k < E; k += kPlanThreads) {
+      const int e = s.order[k];
+      const int h0 = div_small(e, a.inv_eh);
+      const int base = h0 * a.cap + s.cu[h0 * (G + 1) + (e - h0 * Eh)];
+      const int h = s.hoff[e];
+      int run = 0;
+      for (int i = 0; i < P; ++i) {
+        const int d = s.cnt[i * E + e];
+        a.seg[int64_t(i) * a.seg_width + h] = make_int2(d, base + run);
+        cost_part += (long long)cost_a(i, h0, a.gpn, a.inv_gpn) * d;
+        run += d;
+      }
+    }
+  }
   cost_part = warp_sum64(cost_part);
   if (lane == 0) atomicAdd(&s_cost, (unsigned long long)cost_part);
   __syncthreads();
@@ -892,7 +965,7 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
   __syncthreads();
   // exclusive prefix: earlier chunks of this source, then earlier warps
   for (int e = tid; e < E; e += kChunkThreads) {
-    int run = strided_sum(a.chunk_hist + int64_t(il) * a.nchunk * (E + 1) + e, c, E + 1);
+    int run = strided_sum<16>(a.chunk_hist + int64_t(il) * a.nchunk * (E + 1) + e, c, E + 1);
 #pragma unroll
     for (int w = 0; w < kAssignWarps; ++w) {
       const int v = wh[w][e];

@@ -85,6 +85,8 @@ zb::PlanArgs plan_args(const zb_config* c, const zb::Workspace& w, const int32_t
   a.repair = c->repair;
   a.cfix = c->relax ? int(std::floor(double(c->C) * 1048576.0)) : 0;
   a.nchunk = w.nchunk; a.seg_width = w.seg_width;
+  a.inv_gpn = 1.0f / float(c->gpus_per_node);
+  a.inv_eh = 1.0f / float(a.Eh);
   a.ids = ids;
   a.placement = placement;
   if (plan) {

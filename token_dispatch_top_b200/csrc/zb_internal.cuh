@@ -74,6 +74,7 @@ struct PlanArgs {
   int relax, cfix;  // eq. (1)'s band: C as floor(C * 2^20), 0 unless relax
   int repair;       // quota repair between rank pairs after the greedy
   int nchunk, seg_width;
+  float inv_gpn, inv_eh;  // 1/gpn and 1/Eh, for div_small
   int src0;
   int plan_nchunk;
   const int32_t* plan_hist;
