@@ -17,6 +17,9 @@ traffic.  Inputs are seeded and synthetic.
   through buffers larger than L2.
 * ``serial``: the same steps one at a time, L2 flushed before each (outside
   the events) by a 256 MB write and a 256 MB read; per-kernel event times.
+  A bounded device spin (about 0.1 ms) precedes each step, so that the host
+  has enqueued the step's kernels before its first event: the events time
+  the device's latency, not the host's launch overhead.
 * ``e2e``: the same metric through the public API with pinned host buffers:
   each step copies ids, weights and hidden rows host->device, runs the path,
   and copies the combined rows and the plan status back; the copies run on
@@ -57,6 +60,7 @@ METRIC = "plan+dispatch+combine tokens/s at 1 GPU; achieved HBM GB/s vs B200 pea
 UNIT = "tokens/s"
 WORKLOAD = "mid"
 FALLBACK_HBM_GBS = 6650.0
+SLEEP_CYCLES = 200_000  # ~0.1 ms at 1.965 GHz: longer than the host needs to enqueue a step
 
 
 def workload_desc(wl) -> str:
@@ -305,6 +309,7 @@ def measure_workload(wl, dev, flush_l2, peak, iters=10, steps=(0,)):
     for it in range(3 + iters):
         ids, w = inputs[it % len(inputs)]
         flush_l2()
+        torch.cuda._sleep(SLEEP_CYCLES)  # time the device, not the host's launches
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
         ev[0].record(stream)
         zb.plan(plan, ids)
@@ -384,6 +389,12 @@ def run_ours(args, wl, rank, world, local_rank):
 
     stream = torch.cuda.current_stream()
 
+    def hold_device():
+        # keep the device busy (a bounded spin, about 0.1 ms) while the host
+        # enqueues the step that follows, so that its events time the
+        # device's work and not the host's launch overhead
+        torch.cuda._sleep(SLEEP_CYCLES)
+
     def step():
         zb.plan(plan, ids)
         zb.dispatch(plan, hidden, buf)
@@ -411,6 +422,7 @@ def run_ours(args, wl, rank, world, local_rank):
     barrier()
     for k in range(args.steps):
         flush_l2()
+        hold_device()
         ev[k][0].record(stream)
         zb.plan(plan, ids)
         ev[k][1].record(stream)
@@ -503,6 +515,7 @@ def run_ours(args, wl, rank, world, local_rank):
     m_ms, d_ms = [], []
     for _ in range(max(20, min(args.steps, 100))):
         flush_l2()
+        hold_device()
         a0, a1, a2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
         a0.record(stream)
         zb.merge(plan, merged)
@@ -524,6 +537,7 @@ def run_ours(args, wl, rank, world, local_rank):
     cr_ms, cm_ms = [], []
     for _ in range(max(20, min(args.steps, 100))):
         flush_l2()
+        hold_device()
         a0, a1, a2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
         a0.record(stream)
         zb.combine_reduce(plan, merged, buf, w, part)
@@ -544,6 +558,7 @@ def run_ours(args, wl, rank, world, local_rank):
     b_ms = []
     for _ in range(max(20, min(args.steps, 100))):
         flush_l2()
+        hold_device()
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record(stream)
         zb.plan(plan_b, ids)
@@ -580,6 +595,7 @@ def run_ours(args, wl, rank, world, local_rank):
         r_ms = []
         for _ in range(max(20, min(args.steps, 100))):
             flush_l2()
+            hold_device()
             a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a0.record(stream)
             zb.plan_placed(plan_r, ids, pl_d)
@@ -728,7 +744,8 @@ def run_ours(args, wl, rank, world, local_rank):
                        "note": "in the pipelined loop; the plan overlaps the previous "
                                "step's rows"},
         "serial": {"what": "one step at a time on one stream, L2 flushed before each "
-                           "(outside the timing): the latency of an invocation",
+                           "(outside the timing), its kernels enqueued before it starts: "
+                           "the device latency of an invocation",
                    "ms_per_step": serial_ms / args.steps,
                    "value": weak_scaling_value(wl.tokens, world, serial_ms, args.steps),
                    "kernels_ms": {"plan": s_plan_ms / args.steps,

@@ -58,7 +58,7 @@ __device__ __forceinline__ int strided_sum(const int32_t* col, int n, int64_t st
   for (int c = 0; c < n; c += kInFlight) {
     int x[kInFlight];
 #pragma unroll
-    for (int u = 0; u < kInFlight; ++u) x[u] = c + u < n ? col[int64_t(c + u) * stride] : 0;
+    for (int u = 0; u < kInFlight; ++u) x[u] = c + u < n ? __ldcg(col + int64_t(c + u) * stride) : 0;
 #pragma unroll
     for (int u = 0; u < kInFlight; ++u) v += x[u];
   }
@@ -665,10 +665,11 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
   PlannerSmem s = carve(smem_raw, a);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int P = a.P, E = a.E, R = a.R, Eh = a.Eh, G = Eh + R;
-  // the assignment CTAs may launch now (they read their ids before waiting
-  // for this plan); the chunk histograms are read once k_hist has completed
-  griddep_launch_dependents();
+  // the chunk histograms are read once k_hist has completed; from then on
+  // the assignment CTAs may launch (they read their ids and the chunk
+  // histograms before waiting for this plan)
   griddep_wait();
+  griddep_launch_dependents();
 
   // route counts cnt[i][e] (and ids outside [0, E)) summed over the chunks
   if (tid == 0) {
@@ -765,8 +766,10 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
     if (lane < P)
       for (int e = lane * Eh; e < (lane + 1) * Eh; ++e) L += s.hq[e];
     if (lane < P) a.load_before[lane] = L;
-    const long long total = warp_sum64(lane < P ? (long long)L : 0ll);
-    const int T = int((total + P - 1) / P);
+    // sum_r L_r = P*S*K (or the exchanged rows' total), which the validation
+    // keeps below 2^31: 32-bit arithmetic suffices
+    const int total = int(__reduce_add_sync(kFull, lane < P ? unsigned(L) : 0u));
+    const int T = (total + P - 1) / P;
     if (lane == 0) s.misc[kMiscT] = T;
     if (kMode == 2) {
       const int load = greedy_placed_warp(a, s, T, L, lane);
@@ -925,9 +928,10 @@ constexpr int kPerWarp = kChunk / kAssignWarps;  // kPerThread steps of 32
 
 // One CTA per (chunk c, source rank i).  Warp w owns entries
 // [kPerWarp*w, kPerWarp*(w+1)) of the chunk and walks them 32 at a time in flat
-// order, so ranks among equal experts come out in flat-index order.  The ids
-// and their per-warp histograms depend on nothing the plan writes, so they
-// are done while the planner still runs; the rest waits for it.
+// order, so ranks among equal experts come out in flat-index order.  The ids,
+// their per-warp histograms and the prefix over earlier chunks depend on
+// nothing the planner writes, so they are done while the planner still runs;
+// the rest waits for it.
 __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
   __shared__ int32_t wh[kAssignWarps][kMaxE];  // per-warp running position
   __shared__ int32_t s_hoff[kMaxE + 1];
@@ -956,14 +960,10 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
     const unsigned peers = __match_any_sync(kFull, e);
     if (e >= 0 && lane == __ffs(peers) - 1) wh[warp][e] += __popc(peers);
   }
-
-  griddep_wait();  // the planner has completed: its tables are visible
-  if (a.stats[ZB_STAT_STATUS] < 0) return;  // bad ids or capacity: no rows
-  for (int e = tid; e <= E; e += kChunkThreads) s_hoff[e] = a.hoff[e];
-  const int2* segrow = a.seg + int64_t(i) * a.seg_width;
-  for (int x = tid; x < a.seg_width; x += kChunkThreads) s_seg[x] = segrow[x];
   __syncthreads();
-  // exclusive prefix: earlier chunks of this source, then earlier warps
+  // exclusive prefix: earlier chunks of this source, then earlier warps.  The
+  // chunk histograms are complete: the planner launches this kernel only
+  // after its own wait on k_hist has returned.
   for (int e = tid; e < E; e += kChunkThreads) {
     int run = strided_sum<16>(a.chunk_hist + int64_t(il) * a.nchunk * (E + 1) + e, c, E + 1);
 #pragma unroll
@@ -973,7 +973,15 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
       run += v;
     }
   }
+
+  griddep_wait();  // the planner has completed: its tables are visible
+  // the plan's status and the tables this chunk reads, fetched together
+  const int64_t status = a.stats[ZB_STAT_STATUS];
+  for (int e = tid; e <= E; e += kChunkThreads) s_hoff[e] = a.hoff[e];
+  const int2* segrow = a.seg + int64_t(i) * a.seg_width;
+  for (int x = tid; x < a.seg_width; x += kChunkThreads) s_seg[x] = segrow[x];
   __syncthreads();
+  if (status < 0) return;  // bad ids or capacity: no rows
   // pass 2: stable position of each entry, then its segment and row
   const int64_t nrows = int64_t(a.P) * a.cap;
 #pragma unroll
