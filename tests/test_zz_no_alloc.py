@@ -82,7 +82,7 @@ def test_noalloc_band_and_repair(lib, cuda_device):
 def test_noalloc_at_the_size_limit(lib, cuda_device):
     """A config whose workspace is exactly the scratch array's size: the whole
     array, its last bytes included, is usable, and the plan matches zb_plan."""
-    cfg = zb.Config(P=8, E=64, K=8, S=515584, H=8, R=1, cap_rows=2 * 515584 * 8)
+    cfg = zb.Config(P=16, E=176, K=8, S=93952, H=8, R=1, cap_rows=2 * 93952 * 8)
     assert zb.workspace_bytes(cfg) == NOALLOC_SCRATCH_BYTES
     g = torch.Generator(device=cuda_device)
     g.manual_seed(5)
@@ -90,7 +90,7 @@ def test_noalloc_at_the_size_limit(lib, cuda_device):
                         dtype=torch.int32)
     _compare_with_zb_plan(lib, cfg, ids, cuda_device)
     # one more entry per rank needs more scratch than the array holds
-    over = zb.Config(P=8, E=64, K=8, S=515584 + 256, H=8, R=1)
+    over = zb.Config(P=16, E=176, K=8, S=93952 + 256, H=8, R=1)
     assert zb.workspace_bytes(over) > NOALLOC_SCRATCH_BYTES
     plan = zb._Plan(*([256] * 10))
     assert lib.zb_plan_noalloc(ctypes.byref(over.c()), 256, ctypes.byref(plan), None) == \

@@ -1,5 +1,7 @@
 // plan_kernels.cu -- steps 1-3 of an invocation on one GPU:
-//   k_hist     per-(source rank, chunk) expert histogram in shared memory
+//   k_zero     zeroes the per-source totals (one GPU, the plan's first kernel)
+//   k_hist     per-(source rank, chunk) expert histogram in shared memory,
+//              added into the source's totals when there are totals
 //   k_planner  one CTA: route counts, water level, greedy replica placement
 //              (one warp, lanes = ranks; or the quotas over a kept
 //              placement), optional quota repair between rank pairs, quotas,
@@ -148,6 +150,22 @@ __global__ void __launch_bounds__(kChunkThreads) k_hist(PlanArgs a) {
   __syncthreads();
   int32_t* out = a.chunk_hist + (int64_t(i) * a.nchunk + c) * (E + 1);
   for (int e = tid; e <= E; e += kChunkThreads) out[e] = sh[e];
+  if (a.tot) {
+    // the source's totals: zeroed by k_zero, this kernel's predecessor
+    griddep_wait();
+    int32_t* tot = a.tot + int64_t(i) * (E + 1);
+    for (int e = tid; e <= E; e += kChunkThreads)
+      if (sh[e]) atomicAdd(tot + e, sh[e]);
+  }
+}
+
+// Zeroes the per-source totals k_hist adds into (the first kernel of a plan
+// on one GPU; k_hist, launched as its programmatic dependent, histograms its
+// chunk before waiting for it).
+__global__ void __launch_bounds__(kChunkThreads) k_zero(PlanArgs a, int n) {
+  griddep_launch_dependents();
+  const int x = blockIdx.x * kChunkThreads + threadIdx.x;
+  if (x < n) a.tot[x] = 0;
 }
 
 // The count row of one source, counts[e] = sum over its chunks of
@@ -1109,6 +1127,14 @@ cudaError_t launch_hist(const PlanArgs& a, int nsrc, cudaStream_t s) {
   if (a.nchunk == 0 || nsrc == 0) return cudaSuccess;
   k_hist<<<dim3(a.nchunk, nsrc), kChunkThreads, 0, s>>>(a);
   return cudaGetLastError();
+}
+
+cudaError_t launch_hist_totals(const PlanArgs& a, int nsrc, cudaStream_t s) {
+  const int n = nsrc * (a.E + 1);
+  k_zero<<<(n + kChunkThreads - 1) / kChunkThreads, kChunkThreads, 0, s>>>(a, n);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess || a.nchunk == 0 || nsrc == 0) return err;
+  return launch_pdl(k_hist, dim3(a.nchunk, nsrc), dim3(kChunkThreads), 0, s, a);
 }
 
 cudaError_t launch_count_row(const PlanArgs& a, int32_t* counts, cudaStream_t s) {

@@ -96,6 +96,7 @@ zb::PlanArgs plan_args(const zb_config* c, const zb::Workspace& w, const int32_t
     a.dst_row = plan->dst_row; a.row_src = plan->row_src; a.stats = plan->stats;
   }
   a.chunk_hist = reinterpret_cast<int32_t*>(base + w.off_chunk_hist);
+  a.tot = nullptr;
   a.hoff = reinterpret_cast<int32_t*>(base + w.off_hoff);
   a.seg = reinterpret_cast<int2*>(base + w.off_seg);
   a.src0 = 0;
@@ -117,13 +118,17 @@ int plan_impl(const zb_config* c, const int32_t* ids, const int32_t* placement,
   if (!workspace_ok(ws, ws_bytes, w.bytes)) return ZB_ERR_INVALID;
   if (c->S > 0 && !ids) return ZB_ERR_INVALID;
   cudaStream_t s = as_stream(stream);
-  const zb::PlanArgs a = plan_args(c, w, ids, placement, plan, ws);
+  zb::PlanArgs a = plan_args(c, w, ids, placement, plan, ws);
+  // the planner reads the per-source totals that k_hist adds up
+  a.tot = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + w.off_tot);
+  a.plan_hist = a.tot;
+  a.plan_nchunk = 1;
 
   if (a.row_src &&
       cudaMemsetAsync(a.row_src, 0xff, sizeof(int32_t) * size_t(c->P) * c->cap_rows, s) !=
           cudaSuccess)
     return ZB_ERR_CUDA;
-  if (zb::launch_hist(a, c->P, s) != cudaSuccess) return ZB_ERR_CUDA;
+  if (zb::launch_hist_totals(a, c->P, s) != cudaSuccess) return ZB_ERR_CUDA;
   if (zb::launch_planner(a, zb::planner_smem_bytes(*c), s) != cudaSuccess) return ZB_ERR_CUDA;
   if (zb::launch_assign(a, c->P, s) != cudaSuccess) return ZB_ERR_CUDA;
   return ZB_OK;

@@ -33,6 +33,8 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 //                                      sources histogrammed here (all P on one
 //                                      GPU, or one rank's own); column E
 //                                      counts the chunk's ids outside [0, E)
+//   tot        int32 [nsrc][E+1]       the same summed over the chunks (zeroed
+//                                      by k_zero, then added to by k_hist)
 //   hoff       int32 [E+1]             first segment of expert e in a row of seg
 //   seg        int2  [P][E + P*R]      per (source i, expert e): the hosts in
 //                                      the order source i fills them, as
@@ -40,7 +42,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct Workspace {
   int nchunk;
   int seg_width;
-  size_t off_chunk_hist, off_hoff, off_seg, bytes;
+  size_t off_chunk_hist, off_tot, off_hoff, off_seg, bytes;
 };
 
 inline Workspace workspace_layout(const zb_config& c, int nsrc) {
@@ -51,6 +53,8 @@ inline Workspace workspace_layout(const zb_config& c, int nsrc) {
   size_t o = 0;
   w.off_chunk_hist = o;
   o = align256(o + sizeof(int32_t) * size_t(nsrc) * w.nchunk * (c.E + 1));
+  w.off_tot = o;
+  o = align256(o + sizeof(int32_t) * size_t(nsrc) * (c.E + 1));
   w.off_hoff = o;
   o = align256(o + sizeof(int32_t) * size_t(c.E + 1));
   w.off_seg = o;
@@ -62,9 +66,9 @@ inline Workspace workspace_layout(const zb_config& c, int nsrc) {
 // Kernel parameter block shared by the plan kernels.
 //
 // The planner reads the route counts from plan_hist [P][plan_nchunk][E+1],
-// summing each column over its chunks: the per-chunk histograms of every
-// source (whole batch on one GPU), or the exchanged count rows of P ranks
-// (plan_nchunk = 1).  k_hist and k_assign handle the sources src0 ..
+// summing each column over its chunks: the per-source totals k_hist adds up
+// (whole batch on one GPU), or the exchanged count rows of P ranks (both
+// with plan_nchunk = 1).  k_hist and k_assign handle the sources src0 ..
 // src0 + gridDim.y - 1; ids, dst_row and chunk_hist are indexed from src0
 // (local), seg and row_src by the global source.  own_hist, when set, holds
 // the per-chunk histograms of source src0 alone, which the planner checks
@@ -92,6 +96,7 @@ struct PlanArgs {
   int32_t* row_src;
   int64_t* stats;
   int32_t* chunk_hist;
+  int32_t* tot;  // [nsrc][E+1] per-source totals k_hist adds into, or nullptr
   int32_t* hoff;
   int2* seg;
 };
@@ -155,6 +160,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 size_t planner_smem_bytes(const zb_config& c);
 
 cudaError_t launch_hist(const PlanArgs& a, int nsrc, cudaStream_t s);
+cudaError_t launch_hist_totals(const PlanArgs& a, int nsrc, cudaStream_t s);
 cudaError_t launch_count_row(const PlanArgs& a, int32_t* counts, cudaStream_t s);
 cudaError_t launch_planner(const PlanArgs& a, size_t smem, cudaStream_t s);
 cudaError_t launch_assign(const PlanArgs& a, int nsrc, cudaStream_t s);
