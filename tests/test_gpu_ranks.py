@@ -302,3 +302,24 @@ def test_rank_group_one_gpu(dev):
     ok = q.get(timeout=300)
     p.join(timeout=120)
     assert p.exitcode == 0 and ok
+
+
+def test_capacity_on_every_rank_writes_nothing(dev):
+    """A plan whose rows do not fit cap_rows is ZB_ERR_CAPACITY on every rank
+    alike (all ranks compute the same tables), and no rank writes a row."""
+    ids = np.array([[0, 1, 2], [0, 1, 2]], np.int32).reshape(2, 3, 1)
+    kw = dict(P=2, E=6, K=1, S=3, H=16, R=1, cap_rows=3)
+    zc, oc = zb.Config(**kw), oracle.Config(**kw)
+    rps, table, status = _rank_plans(zc, ids, dev)
+    assert status == [zb.ERR_CAPACITY] * 2
+    for r in range(2):
+        assert oracle.plan_rank(oc, r, table, ids[r])["status"] == oracle.ERR_CAPACITY
+    bufs = [torch.full((3, 16), parity.SENTINEL, dtype=torch.int16, device=dev)
+            .view(torch.bfloat16) for _ in range(2)]
+    out = torch.full((3, 16), parity.SENTINEL, dtype=torch.int16, device=dev).view(torch.bfloat16)
+    for r in range(2):
+        zb.dispatch_rank(rps[r], torch.randn((3, 16), device=dev).to(torch.bfloat16), bufs)
+        zb.combine_rank(rps[r], bufs, torch.ones((3, 1), device=dev), out)
+    torch.cuda.synchronize()
+    assert all(bool((b.view(torch.int16) == parity.SENTINEL).all()) for b in bufs)
+    assert bool((out.view(torch.int16) == parity.SENTINEL).all())
