@@ -117,7 +117,9 @@ __device__ __forceinline__ int cost_a(int i, int j, int gpn, float inv_gpn) {
 
 // One CTA per (chunk c, source rank i).  Thread t handles entries
 // t + kChunkThreads*u, u < kPerThread, all loaded before the first is counted.
-// Column E of the chunk's row counts ids outside [0, E).
+// Column E of the chunk's row counts ids outside [0, E).  Each entry is one
+// shared-memory atomic; merging equal ids first with a match-any vote measured
+// slower, most of all on skewed batches (2.4 against 6.0 us on the hot one).
 __global__ void __launch_bounds__(kChunkThreads) k_hist(PlanArgs a) {
   __shared__ int32_t sh[kMaxE + 1];
   griddep_launch_dependents();  // the planner may launch now and wait for us
@@ -142,8 +144,7 @@ __global__ void __launch_bounds__(kChunkThreads) k_hist(PlanArgs a) {
     const int e = ids[u];
     const bool ok = t < n && e >= 0 && e < E;
     bad += (t < n && !ok);
-    const unsigned peers = __match_any_sync(kFull, ok ? e : -1);
-    if (ok && lane == __ffs(peers) - 1) atomicAdd(&sh[e], __popc(peers));
+    if (ok) atomicAdd(&sh[e], 1);
   }
   bad = int(__reduce_add_sync(kFull, unsigned(bad)));
   if (lane == 0 && bad) atomicAdd(&sh[E], bad);
@@ -216,7 +217,8 @@ enum {
   kMiscT = 0, kMiscMax = 1, kMiscNrep = 2, kMiscIters = 3, kMiscBad = 4, kMiscErr = 5,
   kMiscRecv = 6,      // banded plans: the most rows any rank receives
   kMiscRepaired = 7,  // rows moved by quota repair, per direction
-  kMiscNRepExp = 8    // experts with at least one replica (first in order)
+  kMiscNRepExp = 8,   // experts with at least one replica (first in order)
+  kMiscNextRep = 9    // next replicated expert a transport warp takes
 };
 
 // Greedy replica placement, run by one warp; lane r holds rank r's load,
@@ -694,6 +696,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
     s.misc[kMiscBad] = 0;
     s.misc[kMiscErr] = 0;
     s.misc[kMiscRepaired] = 0;
+    s.misc[kMiscNextRep] = 0;
     s_cost = 0ull;
   }
   __syncthreads();
@@ -895,15 +898,24 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
   const bool capacity = rows_max > a.cap;
   long long cost_part = 0;
   if (!capacity) {
-    // experts with replicas: the transport of eq. (1), one warp each
+    // experts with replicas: the transport of eq. (1), one warp each; a warp
+    // takes the next expert when it is done with one, so that experts with
+    // many sources or hosts do not leave the other warps idle
     const int nrx = s.misc[kMiscNRepExp];
-    for (int k = warp; k < nrx; k += kPlanWarps)
+    for (;;) {
+      int k = 0;
+      if (lane == 0) k = atomicAdd(&s.misc[kMiscNextRep], 1);
+      k = __shfl_sync(kFull, k, 0);
+      if (k >= nrx) break;
       cost_part += transport_warp<kBand, true>(a, s, s.order[k], lane, Mw, qw);
+    }
     // experts served by their home rank alone: every source sends it all its
     // rows, one segment per source; a thread per expert walks the sources
     // in rank order (the same segments transport_warp's home-only case
-    // writes, without a warp scan per expert)
-    for (int k = nrx + tid; k < E; k += kPlanThreads) {
+    // writes, without a warp scan per expert).  Threads take them from the
+    // top of the block down: the replicated experts above tend to go to the
+    // warps that reach the counter first, most often the low ones.
+    for (int k = nrx + (kPlanThreads - 1 - tid); k < E; k += kPlanThreads) {
       const int e = s.order[k];
       const int h0 = div_small(e, a.inv_eh);
       const int base = h0 * a.cap + s.cu[h0 * (G + 1) + (e - h0 * Eh)];
