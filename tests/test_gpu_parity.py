@@ -367,6 +367,37 @@ def test_bad_ids_write_nothing(dev):
     assert bool((out.view(torch.int16) == parity.SENTINEL).all())
 
 
+def test_ids_far_out_of_range(dev):
+    """Ids far outside [0, E) (beyond every table an id indexes) are counted
+    and stop the plan like any bad id; the same on the per-rank entry points.
+    A ragged chunk tail follows the bad ids."""
+    rng = np.random.default_rng(11)
+    P, E, K, S = 3, 12, 4, 700
+    ids = rng.integers(0, E, (P, S, K)).astype(np.int32)
+    bad = [(0, 5, 1, 1 << 30), (1, 699, 3, 4096), (2, 0, 0, -7), (2, 321, 2, -(1 << 31)),
+           (1, 100, 0, 384), (0, 600, 2, 2**31 - 1)]
+    for r, t, k, v in bad:
+        ids[r, t, k] = v
+    kw = dict(P=P, E=E, K=K, S=S, H=16, R=1)
+    zc, oc = zb.Config(**kw), oracle.Config(**kw)
+    o = oracle.plan(oc, ids, want_M=False)
+    assert o["status"] == oracle.ERR_BAD_ID
+    p, status, _ = gpu_plan(zc, ids, dev)
+    assert status == oracle.ERR_BAD_ID
+    assert int(p.stats[zb.STAT_BAD_IDS]) == len(bad)
+    rps = [zb.RankPlan(zc, r, dev) for r in range(P)]
+    ids_d = [torch.from_numpy(np.ascontiguousarray(ids[r])).to(dev) for r in range(P)]
+    for r in range(P):
+        zb.count(rps[r], ids_d[r])
+    table = torch.stack([rp.counts for rp in rps])
+    np.testing.assert_array_equal(table.cpu().numpy(),
+                                  np.stack([oracle.count(oc, ids[r]) for r in range(P)]))
+    for r in range(P):
+        rps[r].table.copy_(table)
+        zb.plan_rank(rps[r], ids_d[r])
+        assert int(rps[r].stats[zb.STAT_STATUS]) == oracle.ERR_BAD_ID
+
+
 def test_capacity_then_unbalanced(dev):
     ids = np.array([[0, 1, 2], [0, 1, 2]], np.int32).reshape(2, 3, 1)
     zc = zb.Config(P=2, E=6, K=1, S=3, H=16, R=1, cap_rows=3)

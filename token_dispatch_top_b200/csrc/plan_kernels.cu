@@ -958,12 +958,13 @@ constexpr int kPerWarp = kChunk / kAssignWarps;  // kPerThread steps of 32
 
 // One CTA per (chunk c, source rank i).  Warp w owns entries
 // [kPerWarp*w, kPerWarp*(w+1)) of the chunk and walks them 32 at a time in flat
-// order, so ranks among equal experts come out in flat-index order.  The ids,
-// their per-warp histograms and the prefix over earlier chunks depend on
-// nothing the planner writes, so they are done while the planner still runs;
-// the rest waits for it.
+// order, so ranks among equal experts come out in flat-index order.  Each
+// entry's rank within the source's entries of its expert (earlier chunks,
+// earlier warps, the warp's earlier slices, lower lanes) depends on nothing
+// the planner writes, so it is complete before the wait; after it only the
+// segment lookup and the stores remain.
 __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
-  __shared__ int32_t wh[kAssignWarps][kMaxE];  // per-warp running position
+  __shared__ int32_t wh[kAssignWarps][kMaxE];  // per-warp counts, then bases
   __shared__ int32_t s_hoff[kMaxE + 1];
   __shared__ int2 s_seg[kMaxSegWidth];
   const int c = blockIdx.x, il = blockIdx.y, i = a.src0 + il, tid = threadIdx.x,
@@ -974,21 +975,30 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
   const int n = (nk - start) < kChunk ? int(nk - start) : kChunk;
   const int32_t* src = a.ids + int64_t(il) * nk + start;
   const int w0 = warp * kPerWarp;
+  // ids outside [0, E) become -1 here: they are counted by k_hist and stop
+  // the plan (ZB_ERR_BAD_ID) before any row is written, and no table below
+  // is indexed by them
   int ids[kPerThread];
 #pragma unroll
   for (int u = 0; u < kPerThread; ++u) {
     const int t = w0 + 32 * u + lane;
-    ids[u] = t < n ? __ldg(src + t) : -1;
+    const int v = t < n ? __ldg(src + t) : -1;
+    ids[u] = unsigned(v) < unsigned(E) ? v : -1;
   }
   for (int x = tid; x < kAssignWarps * kMaxE; x += kChunkThreads) (&wh[0][0])[x] = 0;
   __syncthreads();
 
-  // pass 1: per-warp histogram of the warp's slice
+  // pass 1: each entry's rank among the warp's entries of its expert so far,
+  // and the per-warp histogram
+  int pos[kPerThread];
 #pragma unroll
   for (int u = 0; u < kPerThread; ++u) {
     const int e = ids[u];
     const unsigned peers = __match_any_sync(kFull, e);
+    pos[u] = e >= 0 ? wh[warp][e] + __popc(peers & ((1u << lane) - 1u)) : 0;
+    __syncwarp();
     if (e >= 0 && lane == __ffs(peers) - 1) wh[warp][e] += __popc(peers);
+    __syncwarp();
   }
   __syncthreads();
   // exclusive prefix: earlier chunks of this source, then earlier warps.  The
@@ -1003,6 +1013,10 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
       run += v;
     }
   }
+  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < kPerThread; ++u)
+    if (ids[u] >= 0) pos[u] += wh[warp][ids[u]];
 
   griddep_wait();  // the planner has completed: its tables are visible
   // the plan's status and the tables this chunk reads, fetched together
@@ -1012,33 +1026,27 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
   for (int x = tid; x < a.seg_width; x += kChunkThreads) s_seg[x] = segrow[x];
   __syncthreads();
   if (status < 0) return;  // bad ids or capacity: no rows
-  // pass 2: stable position of each entry, then its segment and row
+  // pass 2: each entry's segment (the host its rank falls in) and row
   const int64_t nrows = int64_t(a.P) * a.cap;
 #pragma unroll
   for (int u = 0; u < kPerThread; ++u) {
     const int e = ids[u];
-    const unsigned peers = __match_any_sync(kFull, e);
-    int p = 0;
-    if (e >= 0) p = wh[warp][e] + __popc(peers & ((1u << lane) - 1u));
-    __syncwarp();
-    if (e >= 0 && lane == __ffs(peers) - 1) wh[warp][e] += __popc(peers);
-    __syncwarp();
-    if (e >= 0) {
-      const int h_end = s_hoff[e + 1];
-      int prev = 0, row = -1;
-      for (int h = s_hoff[e]; h < h_end; ++h) {
-        const int2 sg = s_seg[h];
-        if (p < sg.x) {
-          row = sg.y + (p - prev);
-          break;
-        }
-        prev = sg.x;
+    if (e < 0) continue;
+    const int p = pos[u];
+    const int h_end = s_hoff[e + 1];
+    int prev = 0, row = -1;
+    for (int h = s_hoff[e]; h < h_end; ++h) {
+      const int2 sg = s_seg[h];
+      if (p < sg.x) {
+        row = sg.y + (p - prev);
+        break;
       }
-      const int64_t f = start + w0 + 32 * u + lane;
-      a.dst_row[int64_t(il) * nk + f] = row;
-      if (a.row_src && row >= 0 && int64_t(row) < nrows)
-        a.row_src[row] = int32_t(int64_t(i) * nk + f);
+      prev = sg.x;
     }
+    const int64_t f = start + w0 + 32 * u + lane;
+    a.dst_row[int64_t(il) * nk + f] = row;
+    if (a.row_src && row >= 0 && int64_t(row) < nrows)
+      a.row_src[row] = int32_t(int64_t(i) * nk + f);
   }
 }
 
