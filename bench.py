@@ -32,6 +32,10 @@ traffic.  Inputs are seeded and synthetic.
 * ``extras.workloads`` (N=1): the other four workloads one invocation at a
   time: plan latency, dispatch and combine rates and fractions of the peak,
   and the plan's balance (drift: steps 0, 31 and 63).
+* ``extras.rank_path`` (N=1): the entry points one rank of P GPUs calls
+  (count, plan_rank, dispatch_rank, combine_rank) for each of the P ranks of
+  the same workload in turn, each call timed alone; checked against the
+  whole-batch path's rows.
 
 With ``--impl reference`` the CPU oracle itself is timed on the same workload
 (rank 0 only; other ranks exit).  With N>1 (torchrun), every rank runs an
@@ -63,6 +67,13 @@ FALLBACK_HBM_GBS = 6650.0
 SLEEP_CYCLES = 200_000  # ~0.1 ms at 1.965 GHz: longer than the host needs to enqueue a step
 
 
+def route_steps(wl) -> tuple:
+    """The routing steps a run cycles through: step 0 alone, or, for a workload
+    that drifts over many steps, 8 of them spread over the walk (a new draw,
+    and so a new plan, at every timed step)."""
+    return tuple(range(0, wl.steps, max(1, wl.steps // 8))) if wl.steps > 1 else (0,)
+
+
 def workload_desc(wl) -> str:
     if wl.hot_share is not None:
         pop = (f"4 hottest experts take {wl.hot_share:.0%} of assignments, the rest Zipf "
@@ -75,8 +86,11 @@ def workload_desc(wl) -> str:
         pop += f", log-popularity random walk sigma={wl.walk_sigma} per step"
     nodes = f", {wl.P // wl.gpus_per_node} nodes x {wl.gpus_per_node}" \
         if wl.gpus_per_node > 1 else ""
+    steps = route_steps(wl)
+    cycle = f"; step k re-plans on walk step {steps[1] - steps[0]}*(k mod {len(steps)})" \
+        if len(steps) > 1 else ""
     return (f"{wl.name}: P={wl.P}{nodes} E={wl.E} K={wl.K} S={wl.S} H={wl.H} R={wl.R} "
-            f"C={wl.C}, {pop}, seed 0")
+            f"C={wl.C}, {pop}, seed 0{cycle}")
 
 
 def config_dict(wl, n_gpus: int) -> dict:
@@ -211,16 +225,21 @@ def weak_scaling_value(tokens_per_rank: int, world: int, total_ms: float, steps:
     return tokens_per_rank * world / (total_ms / steps / 1000.0)
 
 
-def oracle_steps(wl, ids, w, hidden_bits, budget_s: float, min_steps: int = 1):
-    """Full CPU-oracle steps (plan + dispatch + combine) until the budget is spent.
-    Returns (steps, seconds)."""
+def oracle_steps(wl, routes, hidden_bits, budget_s: float, min_steps: int = 1):
+    """Full CPU-oracle steps (plan + dispatch + combine) until the budget is
+    spent, step k on routes[k mod len(routes)] (ids, w).  Returns (steps,
+    seconds)."""
     import oracle
-    cfg = oracle.Config(wl.P, wl.E, wl.K, wl.S, wl.H, wl.R, wl.C, wl.gpus_per_node, None)
+    cfg = oracle.Config(wl.P, wl.E, wl.K, wl.S, wl.H, wl.R, wl.C, wl.gpus_per_node,
+                        data_cap_rows(wl))
     buf = np.empty((wl.P, cfg.cap(), wl.H), np.uint16)
     n = 0
     t0 = time.perf_counter()
     while n < min_steps or time.perf_counter() - t0 < budget_s:
+        ids, w = routes[n % len(routes)]
         p = oracle.plan(cfg, ids, want_M=False)
+        if p["status"] < 0:
+            raise RuntimeError(f"oracle plan failed: status {p['status']}")
         oracle.dispatch(cfg, p["dst_row"], hidden_bits, buf)
         oracle.combine(cfg, p["dst_row"], buf.reshape(-1, wl.H), w)
         n += 1
@@ -252,20 +271,20 @@ def run_reference(args, wl, rank, budget_s: float = 120.0):
         return
     import oracle
     from token_dispatch_top_b200 import synth
-    ids, w = synth.routing(wl, 0)
+    routes = [synth.routing(wl, 0, st) for st in route_steps(wl)]
     hidden = synth.hidden_bits(wl, 0)
     cfg = oracle.Config(wl.P, wl.E, wl.K, wl.S, wl.H, wl.R, wl.C, wl.gpus_per_node,
                         data_cap_rows(wl))
     buf = np.empty((wl.P, cfg.cap(), wl.H), np.uint16)
     probe = min(1024, wl.tokens)
-    tp, td = oracle_sampled_step(wl, cfg, ids, w, hidden, buf, probe)
+    tp, td = oracle_sampled_step(wl, cfg, *routes[0], hidden, buf, probe)
     per_step = budget_s / max(1, args.steps + args.warmup)
     n_tok = int(max(64, min(wl.tokens, probe * (per_step - tp) / max(td, 1e-9))))
-    for _ in range(args.warmup):
-        oracle_sampled_step(wl, cfg, ids, w, hidden, buf, n_tok)
+    for k in range(args.warmup):
+        oracle_sampled_step(wl, cfg, *routes[k % len(routes)], hidden, buf, n_tok)
     t_plan = t_data = 0.0
-    for _ in range(args.steps):
-        a, b = oracle_sampled_step(wl, cfg, ids, w, hidden, buf, n_tok)
+    for k in range(args.steps):
+        a, b = oracle_sampled_step(wl, cfg, *routes[k % len(routes)], hidden, buf, n_tok)
         t_plan += a
         t_data += b
     full_step_s = (t_plan + t_data * wl.tokens / n_tok) / args.steps
@@ -351,6 +370,99 @@ def measure_workload(wl, dev, flush_l2, peak, iters=10, steps=(0,)):
     return rec
 
 
+def measure_rank_path(wl, dev, flush_l2, peak, iters=5):
+    """The form one rank of P GPUs runs, its P ranks one after another on this
+    GPU: per rank, zb.count on its own ids, zb.plan_rank from the stacked
+    count rows (what the all-gather between GPUs yields), and zb.dispatch_rank /
+    zb.combine_rank through the table of P buffer pointers, here P parts of
+    one allocation.  count and plan_rank are timed one call at a time; the
+    P dispatch_rank calls, and then the P combine_rank calls, are timed back
+    to back inside one pair of events, since one call alone (about 25 us on
+    mid) is short beside the events' own overhead.  L2 is flushed before
+    each timed region, outside its events.  Every rank's dst_row and
+    combined rows must equal the whole-batch path's."""
+    import numpy as np
+    import torch
+    from token_dispatch_top_b200 import synth, zb
+    cfg = zb.Config(P=wl.P, E=wl.E, K=wl.K, S=wl.S, H=wl.H, R=wl.R, C=wl.C,
+                    gpus_per_node=wl.gpus_per_node, cap_rows=data_cap_rows(wl))
+    P, S, H, cap = cfg.P, cfg.S, cfg.H, cfg.cap
+    ids_np, w_np = synth.routing(wl, 0)
+    ids_all = torch.from_numpy(ids_np).to(dev)
+    w_all = torch.from_numpy(w_np).to(dev)
+    hidden = synth.hidden_device(wl, 0, 0, dev)
+    ids = [ids_all[r] for r in range(P)]
+    rps = [zb.RankPlan(cfg, r, dev) for r in range(P)]
+    buf = torch.empty((P, cap, H), dtype=torch.bfloat16, device=dev)
+    bufs = list(buf.unbind(0))
+    out = torch.empty((P, S, H), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        flush_l2()
+        torch.cuda._sleep(SLEEP_CYCLES)  # time the device, not the host's launches
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        return a.elapsed_time(b)
+
+    def dispatch_all():
+        for r in range(P):
+            zb.dispatch_rank(rps[r], hidden[r], bufs)
+
+    def combine_all():
+        for r in range(P):
+            zb.combine_rank(rps[r], bufs, w_all[r], out[r])
+
+    t = {"count": [], "plan_rank": [], "dispatch_rank": [], "combine_rank": []}
+    for it in range(1 + iters):
+        tc = [timed(lambda r=r: zb.count(rps[r], ids[r])) for r in range(P)]
+        table = torch.stack([rp.counts for rp in rps])  # the exchange (not timed)
+        for rp in rps:
+            rp.table.copy_(table)
+        tp = [timed(lambda r=r: zb.plan_rank(rps[r], ids[r])) for r in range(P)]
+        for rp in rps:
+            status, _ = zb.plan_status(rp)
+            if status < 0:
+                raise RuntimeError(f"rank plan failed: {zb.strerror(status)}")
+        td = timed(dispatch_all)
+        tk = timed(combine_all)
+        if it >= 1:
+            t["count"].extend(tc)
+            t["plan_rank"].extend(tp)
+            t["dispatch_rank"].append(td)
+            t["combine_rank"].append(tk)
+    # the whole-batch path on the same inputs: the same rows, bit for bit
+    whole = zb.Plan(cfg, dev, with_row_src=False)
+    zb.plan(whole, ids_all)
+    wbuf = torch.empty_like(buf)
+    wout = torch.empty_like(out)
+    zb.dispatch(whole, hidden, wbuf)
+    zb.combine(whole, wbuf, w_all, wout)
+    same = all(torch.equal(rps[r].dst_row, whole.dst_row[r]) for r in range(P)) and \
+        torch.equal(out.view(torch.int16), wout.view(torch.int16))
+    if not same:
+        raise RuntimeError("per-rank path differs from the whole-batch path")
+    ab = algorithmic_bytes(wl)  # summed over the P ranks: the same bytes
+    d, c = statistics.median(t["dispatch_rank"]), statistics.median(t["combine_rank"])
+    rec = {"what": "the per-rank entry points of the P-GPU form, its P ranks run one after "
+                   "another on one GPU, buffers addressed through the P-pointer table; "
+                   "not part of the step",
+           "workload": workload_desc(wl), "iterations": iters,
+           "count_us_per_rank": 1000.0 * statistics.median(t["count"]),
+           "plan_rank_us_per_rank": 1000.0 * statistics.median(t["plan_rank"]),
+           "dispatch_rank": {"ms_all_ranks": d, "gbs": ab["dispatch"] / d / 1e6,
+                             "frac": ab["dispatch"] / d / 1e6 / peak},
+           "combine_rank": {"ms_all_ranks": c, "gbs": ab["combine"] / c / 1e6,
+                            "frac": ab["combine"] / c / 1e6 / peak},
+           "same_rows_as_whole_batch": bool(same)}
+    del rps, buf, bufs, out, wbuf, wout, whole, hidden
+    torch.cuda.empty_cache()
+    return rec
+
+
 def run_ours(args, wl, rank, world, local_rank):
     import torch
     from token_dispatch_top_b200 import build, synth, zb
@@ -365,14 +477,17 @@ def run_ours(args, wl, rank, world, local_rank):
         dist = dist_mod
 
     seed = rank
-    ids_np, w_np = synth.routing(wl, seed)
+    routes_np = [synth.routing(wl, seed, st) for st in route_steps(wl)]
+    n_routes = len(routes_np)
+    ids_np, w_np = routes_np[0]
     hidden_np = synth.hidden_bits(wl, seed)
     cfg = zb.Config(P=wl.P, E=wl.E, K=wl.K, S=wl.S, H=wl.H, R=wl.R, C=wl.C,
                     gpus_per_node=wl.gpus_per_node, cap_rows=data_cap_rows(wl))
     P, S, K, H, cap = cfg.P, cfg.S, cfg.K, cfg.H, cfg.cap
 
-    ids = torch.from_numpy(ids_np).to(dev)
-    w = torch.from_numpy(w_np).to(dev)
+    ids_l = [torch.from_numpy(a).to(dev) for a, _ in routes_np]
+    w_l = [torch.from_numpy(b).to(dev) for _, b in routes_np]
+    ids, w = ids_l[0], w_l[0]  # the step-0 draw, for the checks and extras
     hidden = torch.from_numpy(hidden_np.view(np.int16)).to(dev).view(torch.bfloat16)
     plan = zb.Plan(cfg, dev, with_row_src=False)
     buf = torch.empty((P, cap, H), dtype=torch.bfloat16, device=dev)
@@ -395,25 +510,26 @@ def run_ours(args, wl, rank, world, local_rank):
         # device's work and not the host's launch overhead
         torch.cuda._sleep(SLEEP_CYCLES)
 
-    def step():
-        zb.plan(plan, ids)
+    def step(k=0):
+        zb.plan(plan, ids_l[k % n_routes])
         zb.dispatch(plan, hidden, buf)
-        zb.combine(plan, buf, w, out)
+        zb.combine(plan, buf, w_l[k % n_routes], out)
 
-    # the plan must balance (status OK) and must fit the S*K buffers
-    step()
-    status, max_load = zb.plan_status(plan)
-    if status < 0:
-        raise RuntimeError(f"plan failed: {zb.strerror(status)}")
+    # every draw's plan must fit the receive buffers
+    for k in range(n_routes):
+        step(k)
+        status, max_load = zb.plan_status(plan)
+        if status < 0:
+            raise RuntimeError(f"plan failed: {zb.strerror(status)}")
 
     def barrier():
         torch.cuda.synchronize()
         if dist is not None:
             dist.barrier()
 
-    for _ in range(args.warmup):
+    for k in range(args.warmup):
         flush_l2()
-        step()
+        step(k)
     barrier()
     n_ev = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_ev)]
@@ -424,11 +540,11 @@ def run_ours(args, wl, rank, world, local_rank):
         flush_l2()
         hold_device()
         ev[k][0].record(stream)
-        zb.plan(plan, ids)
+        zb.plan(plan, ids_l[k % n_routes])
         ev[k][1].record(stream)
         zb.dispatch(plan, hidden, buf)
         ev[k][2].record(stream)
-        zb.combine(plan, buf, w, out)
+        zb.combine(plan, buf, w_l[k % n_routes], out)
         ev[k][3].record(stream)
     barrier()
     status, _ = zb.plan_status(plan)
@@ -465,7 +581,7 @@ def run_ours(args, wl, rank, world, local_rank):
                     s_plan.wait_event(rows_done[sl])  # step k-2 is done with the slot
                 if pev is not None:
                     pev[k][0].record(s_plan)
-                zb.plan(plans2[sl], ids)
+                zb.plan(plans2[sl], ids_l[k % n_routes])
                 if pev is not None:
                     pev[k][1].record(s_plan)
                 plan_done[sl].record(s_plan)
@@ -476,7 +592,7 @@ def run_ours(args, wl, rank, world, local_rank):
                 zb.dispatch(plans2[sl], hidden, bufs2[sl])
                 if pev is not None:
                     pev[k][3].record(s_rows)
-                zb.combine(plans2[sl], bufs2[sl], w, outs2[sl])
+                zb.combine(plans2[sl], bufs2[sl], w_l[k % n_routes], outs2[sl])
                 if pev is not None:
                     pev[k][4].record(s_rows)
                 rows_done[sl].record(s_rows)
@@ -496,8 +612,16 @@ def run_ours(args, wl, rank, world, local_rank):
         st_, _ = zb.plan_status(pl_)
         if st_ < 0:
             raise RuntimeError(f"plan failed in the pipelined loop: {zb.strerror(st_)}")
-    if args.steps >= 2 and not torch.equal(outs2[0].view(torch.int16), outs2[1].view(torch.int16)):
-        raise RuntimeError("the two pipeline slots disagree")
+    # the last step's output against the same step run alone (into an output
+    # of its own: plan, buf and out are pipeline slot 0's)
+    last = args.steps - 1
+    chk = torch.empty_like(out)
+    zb.plan(plan, ids_l[last % n_routes])
+    zb.dispatch(plan, hidden, buf)
+    zb.combine(plan, buf, w_l[last % n_routes], chk)
+    if not torch.equal(outs2[last % 2].view(torch.int16), chk.view(torch.int16)):
+        raise RuntimeError("the pipelined loop's output differs from a serial step")
+    del chk
     step_ms = p_start.elapsed_time(p_end)  # total over K steps
     p_plan = [pev[k][0].elapsed_time(pev[k][1]) for k in range(n_ev)]
     p_disp = [pev[k][2].elapsed_time(pev[k][3]) for k in range(n_ev)]
@@ -614,8 +738,8 @@ def run_ours(args, wl, rank, world, local_rank):
     # run on their own streams with three buffer slots, so one step's input
     # copy overlaps the previous step's output copy (the host link is full
     # duplex); compute stays in order on the compute stream.
-    ids_h = torch.from_numpy(ids_np).pin_memory()
-    w_h = torch.from_numpy(w_np).pin_memory()
+    ids_h = [torch.from_numpy(a).pin_memory() for a, _ in routes_np]
+    w_h = [torch.from_numpy(b).pin_memory() for _, b in routes_np]
     hid_h = torch.from_numpy(hidden_np.view(np.int16)).pin_memory()
     n_slots = 3
     out_h = [torch.empty((P, S, H), dtype=torch.int16).pin_memory() for _ in range(n_slots)]
@@ -643,8 +767,8 @@ def run_ours(args, wl, rank, world, local_rank):
             with torch.cuda.stream(h2d_s):
                 if k >= n_slots:
                     h2d_s.wait_event(comp_done[sl])  # slot's inputs consumed
-                ids_d[sl].copy_(ids_h, non_blocking=True)
-                w_d[sl].copy_(w_h, non_blocking=True)
+                ids_d[sl].copy_(ids_h[k % n_routes], non_blocking=True)
+                w_d[sl].copy_(w_h[k % n_routes], non_blocking=True)
                 hid_d[sl].copy_(hid_h, non_blocking=True)
                 h2d_done[sl].record(h2d_s)
             comp_s.wait_event(h2d_done[sl])
@@ -678,6 +802,8 @@ def run_ours(args, wl, rank, world, local_rank):
     # ---- the other workloads, one invocation at a time (N = 1 only): plan
     # latency, dispatch and combine rates, balance
     workloads = {}
+    rank_path = None
+    event_floor_us = None
     if world == 1 and args.extras:
         peak_gbs, _ = read_peaks()
         torch.cuda.empty_cache()
@@ -687,6 +813,24 @@ def run_ours(args, wl, rank, world, local_rank):
             steps = (0, 31, 63) if name == "drift" else (0,)
             workloads[name] = measure_workload(synth.WORKLOADS[name], dev, flush_l2, peak_gbs,
                                                steps=steps)
+        # the per-rank entry points of the P-GPU form on this workload
+        rank_path = measure_rank_path(wl, dev, flush_l2, peak_gbs)
+        # what the same flush, hold and event pair read around the shortest
+        # kernel there is (a one-element fill): the floor under every plan
+        # latency above
+        one = torch.zeros(1, dtype=torch.int32, device=dev)
+        floor = []
+        for k in range(13):
+            flush_l2()
+            hold_device()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            one.fill_(k)
+            b.record(stream)
+            b.synchronize()
+            if k >= 3:
+                floor.append(a.elapsed_time(b))
+        event_floor_us = 1000.0 * statistics.median(floor)
 
     # ---- max over ranks
     (step_ms, e2e_ms, disp_ms, comb_ms, plan_ms, serial_ms, s_disp_ms, s_comb_ms,
@@ -711,7 +855,7 @@ def run_ours(args, wl, rank, world, local_rank):
 
     cpu = None
     if world == 1:
-        n, sec = oracle_steps(wl, ids_np, w_np, hidden_np, budget_s=10.0)
+        n, sec = oracle_steps(wl, routes_np, hidden_np, budget_s=10.0)
         cpu = {"value": wl.tokens * n / sec, "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": f"{n} full steps (plan+dispatch+combine) of the same workload, "
                          "single-threaded C"}
@@ -771,7 +915,11 @@ def run_ours(args, wl, rank, world, local_rank):
                 "combine_gbs": (rows_merged * wl.H * 2 + wl.N * 4 + wl.tokens * wl.H * 2)
                 / statistics.median(cm_ms) / 1e6},
             "banded_plan": banded, "quota_repair": rep,
-            "workloads": workloads},
+            "workloads": workloads, "rank_path": rank_path,
+            "event_floor_us": {"what": "a one-element fill timed like the plan (L2 flushed, "
+                                       "device held, one event pair): the events' own "
+                                       "floor under plan_latency_us",
+                               "value": event_floor_us}},
         "plan_latency_us": dict({wl.name: 1000.0 * s_plan_ms / args.steps},
                                 **{k: v["plan_us"] for k, v in workloads.items()}),
         "wall_s": wall,
@@ -792,6 +940,8 @@ def main():
     ap.add_argument("--no-extras", dest="extras", action="store_false",
                     help="skip the per-workload records of the other workloads")
     args = ap.parse_args()
+    if args.steps < 1:
+        ap.error("--steps must be at least 1")
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be at least 3")
 

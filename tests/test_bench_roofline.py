@@ -7,6 +7,8 @@
   they were measured on hash to the recorded value, and None for a changed
   source, a missing file or an unknown kernel.
 * the peak comes from the measured peaks file when present.
+* a drifting workload cycles through 8 draws of its walk, and the CPU
+  baseline plans with the same receive buffers as the GPU arm.
 """
 import json
 import os
@@ -64,3 +66,30 @@ def test_peak_from_measured_file(tmp_path, monkeypatch):
     assert bench.read_peaks() == (bench.FALLBACK_HBM_GBS, "fallback")
     (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6508.8}))
     assert bench.read_peaks() == (6508.8, "measured")
+
+
+def test_route_steps_and_the_shared_config():
+    """A drifting workload cycles through 8 draws of its walk; the others use
+    one.  Both arms print the same config dict, which names the cycle."""
+    assert bench.route_steps(synth.WORKLOADS["mid"]) == (0,)
+    drift = synth.WORKLOADS["drift"]
+    assert bench.route_steps(drift) == tuple(range(0, 64, 8))
+    assert "re-plans on walk step 8*(k mod 8)" in bench.config_dict(drift, 1)["workload"]
+    assert bench.config_dict(drift, 2) == bench.config_dict(drift, 2)
+
+
+def test_oracle_steps_use_the_runs_buffers():
+    """The CPU baseline plans with the same receive buffers as the GPU arm:
+    on a workload the slots cannot balance to S*K rows (cap_rows = 2*S*K), a
+    plan at S*K rows would fail and move nothing."""
+    import dataclasses
+    hot = synth.WORKLOADS["hot"]
+    small = dataclasses.replace(hot, S=64, H=64)
+    import oracle
+    routes = [synth.routing(small, 0)]
+    at_sk = oracle.Config(small.P, small.E, small.K, small.S, small.H, small.R, small.C,
+                          small.gpus_per_node, None)
+    assert oracle.plan(at_sk, routes[0][0], want_M=False)["status"] == oracle.ERR_CAPACITY
+    assert bench.data_cap_rows(small) == 2 * small.S * small.K
+    n, sec = bench.oracle_steps(small, routes, synth.hidden_bits(small, 0), budget_s=0.0)
+    assert n == 1 and sec >= 0.0  # the baseline's plan fits (it raises otherwise)
