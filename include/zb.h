@@ -476,6 +476,41 @@ ZB_API int zb_recalibrate(const zb_config *cfg, const int32_t *cnt, int32_t *pla
                           float eps, int max_swaps, void *workspace, size_t workspace_bytes,
                           void *stream, int32_t *swaps, int32_t *max_load);
 
+/* ------------------------------------------------------ bounds-checked build
+ *
+ * Built with -DZB_DEBUG (token_dispatch_top_b200/libzb_debug.so), every
+ * kernel checks the accesses whose index comes from data -- a row number
+ * from dst_row or from the segment table, an expert id, a slot -- against
+ * the extent of what it indexes.  A failed check skips that access and is
+ * recorded on the device: a count, and the site, index and bound of the
+ * first failure.  This stands in for a memory checker: the GPU tests can run
+ * against the debug library and require that nothing was recorded.
+ *
+ * The release library keeps the guards that protect memory (rows outside
+ * [0, P*cap) are skipped) and compiles the rest of the checks away; there,
+ * zb_debug_read returns ZB_ERR_INVALID and touches nothing. */
+#define ZB_SITE_ASSIGN_EXPERT 1 /* k_assign: per-warp histogram indexed by an id */
+#define ZB_SITE_ASSIGN_SEGMENT 2 /* k_assign: segment index from hoff */
+#define ZB_SITE_ASSIGN_ROW 3    /* k_assign: the row an entry is given */
+#define ZB_SITE_PLAN_SEGMENT 4  /* k_planner: segment-table write */
+#define ZB_SITE_PLAN_SLOT 5     /* k_planner / k_eval_placements: helper slot or holder table */
+#define ZB_SITE_DISPATCH_ROW 6  /* k_dispatch*: a destination row of dst_row */
+#define ZB_SITE_COMBINE_ROW 7   /* k_combine*: a source row of dst_row */
+#define ZB_SITE_MERGE_ROW 8     /* merge kernels: a row of dst_row or of the merged layout */
+typedef struct zb_debug_record {
+  uint64_t count; /* failed checks since the last reset, over all kernels */
+  int32_t site;   /* ZB_SITE_* of the first failure recorded (0: none) */
+  int32_t reserved;
+  int64_t index;  /* its index */
+  int64_t bound;  /* and the extent the index had to stay below */
+} zb_debug_record;
+
+/* Copies the record into *out (host) and, when reset != 0, clears it.
+ * Synchronises the device.  ZB_ERR_INVALID in the release library or for a
+ * NULL out; ZB_ERR_CUDA if a CUDA call fails.  The record is per process and
+ * per device; calls from several threads at once are not ordered. */
+ZB_API int zb_debug_read(zb_debug_record *out, int reset);
+
 #ifdef __cplusplus
 }
 #endif

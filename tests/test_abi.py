@@ -38,6 +38,22 @@ def test_exports_match_header(lib):
         assert hasattr(lib, name)
 
 
+def test_debug_library_exports_the_same_and_release_keeps_no_record(lib):
+    """libzb_debug.so (the bounds-checked build) exports what the header
+    declares; zb_debug_read answers ZB_ERR_INVALID in the release library,
+    and for a NULL record in the debug one, before touching a device."""
+    dbg = build.build(debug=True)
+    out = subprocess.check_output(["nm", "-D", "--defined-only", dbg], text=True)
+    exported = sorted(line.split()[-1] for line in out.splitlines()
+                      if line.split()[-1].startswith("zb_"))
+    assert exported == _declared()
+    rec = zb._DebugRecord()
+    release = ctypes.CDLL(build.LIB)
+    assert release.zb_debug_read(ctypes.byref(rec), 1) == zb.ERR_INVALID
+    assert ctypes.CDLL(dbg).zb_debug_read(None, 0) == zb.ERR_INVALID
+    assert ctypes.sizeof(zb._DebugRecord) == 32
+
+
 def test_strerror(lib):
     for code in (zb.OK, zb.WARN_UNBALANCED, zb.ERR_INVALID, zb.ERR_CAPACITY, zb.ERR_BAD_ID,
                  zb.ERR_TIMEOUT, zb.ERR_CUDA, 12345):

@@ -18,6 +18,7 @@
 #include "zb_rows.cuh"
 
 namespace zb {
+ZB_DEBUG_TU(debug_read_merge)
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
@@ -25,13 +26,15 @@ constexpr int kMergeThreads = 256;  // one token per thread
 constexpr int kMergeWarps = kMergeThreads / 32;
 constexpr int kTokPerThread = kMergeChunk / kMergeThreads;  // 1
 
-// Bit j set when one of token t's entries goes to rank j.
+// Bit j set when one of token t's entries goes to rank j (rows outside
+// [0, nrows), which a plan with a non-negative status never holds, count
+// nowhere).
 __device__ __forceinline__ unsigned rank_mask(const int32_t* dst_row, int64_t t, int K,
-                                              int cap) {
+                                              int cap, int64_t nrows) {
   unsigned m = 0u;
   for (int k = 0; k < K; ++k) {
     const int d = __ldg(dst_row + t * K + k);
-    if (d >= 0) m |= 1u << (d / cap);
+    if (ZB_IN(ZB_SITE_MERGE_ROW, d, nrows) && d >= 0 && d < nrows) m |= 1u << (d / cap);
   }
   return m;
 }
@@ -45,7 +48,7 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge_count(MergeArgs a) {
   for (int u = 0; u < kTokPerThread; ++u) {
     const int64_t t = int64_t(c) * kMergeChunk + u * kMergeThreads + tid;
     if (t < a.ntok) {
-      unsigned m = rank_mask(a.dst_row, t, a.K, a.cap);
+      unsigned m = rank_mask(a.dst_row, t, a.K, a.cap, int64_t(a.P) * a.cap);
       while (m) {
         const int j = __ffs(m) - 1;
         m &= m - 1u;
@@ -116,7 +119,10 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge_assign(MergeArgs a) {
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
       if (k >= K) break;
-      if (d[k] < 0 || d[k] >= nrows) continue;  // only a valid plan has rows
+      if (d[k] < 0 || d[k] >= nrows) {  // only a valid plan has rows
+        ZB_FAIL(ZB_SITE_MERGE_ROW, d[k], nrows);
+        continue;
+      }
       const int j = d[k] / cap;
       int pj = 0;
 #pragma unroll
@@ -144,7 +150,8 @@ __global__ void __launch_bounds__(256) k_dispatch_merged(int ntok, int H, int64_
   const int nv = H >> 3;
   const int my = lane < K ? __ldg(tok_row + t * K + lane) : -2 - lane;
   const unsigned peers = __match_any_sync(kFull, my);
-  const bool first = lane < K && (__ffs(peers) - 1) == lane && my >= 0 && my < nrows;
+  const bool in = lane >= K || ZB_IN(ZB_SITE_MERGE_ROW, my, nrows);
+  const bool first = in && lane < K && (__ffs(peers) - 1) == lane && my >= 0 && my < nrows;
   const unsigned firsts = __ballot_sync(kFull, first);
   int64_t rows[K];
 #pragma unroll
@@ -206,6 +213,8 @@ __global__ void __launch_bounds__(256) k_combine_reduce(int ntok, int H, int64_t
     mrow[k] = __shfl_sync(kFull, my_m, k);
     wk[k] = __shfl_sync(kFull, my_w, k);
     ok = ok && r >= 0 && r < nrows && mrow[k] >= 0 && mrow[k] < nrows;
+    if (!(r >= 0 && r < nrows)) ZB_FAIL(ZB_SITE_MERGE_ROW, r, nrows);
+    if (!(mrow[k] >= 0 && mrow[k] < nrows)) ZB_FAIL(ZB_SITE_MERGE_ROW, mrow[k], nrows);
     rows[k] = int64_t(r) * nv;
   }
   if (!ok) return;  // a corrupt plan or layout: write nothing for this token
@@ -259,6 +268,7 @@ __global__ void __launch_bounds__(256) k_combine_merged(int ntok, int H, int64_t
   for (int k = 0; k < K; ++k) {
     const int m = __shfl_sync(kFull, my_m, k);
     ok = ok && m >= 0 && m < nrows;
+    if (!(m >= 0 && m < nrows)) ZB_FAIL(ZB_SITE_MERGE_ROW, m, nrows);
     rows[k] = int64_t(m) * nv;
   }
   if (!ok) return;

@@ -21,26 +21,34 @@
 #include "zb_rows.cuh"
 
 namespace zb {
+ZB_DEBUG_TU(debug_read_move)
 namespace {
 
 constexpr int kMoveThreads = 256;
 constexpr int kMoveWarps = kMoveThreads / 32;
 
+// A row outside [0, P*cap) -- which a plan with a non-negative status never
+// holds -- gives nullptr, and the access is skipped (recorded at `site` in the
+// bounds-checked build).
 struct FlatRows {
   char* base;
   int64_t nrows;  // P * cap
-  __device__ __forceinline__ char* row(int d, int64_t row_bytes) const {
-    return (d >= 0 && d < nrows) ? base + int64_t(d) * row_bytes : nullptr;
+  __device__ __forceinline__ char* row(int d, int64_t row_bytes, int site) const {
+    if (d >= 0 && d < nrows) return base + int64_t(d) * row_bytes;
+    ZB_FAIL(site, d, nrows);
+    return nullptr;
   }
 };
 
 struct RankRows {
   RankBufs t;
   int P, cap;
-  __device__ __forceinline__ char* row(int d, int64_t row_bytes) const {
-    if (d < 0) return nullptr;
-    const int j = d / cap;
-    if (j >= P) return nullptr;
+  __device__ __forceinline__ char* row(int d, int64_t row_bytes, int site) const {
+    const int j = d >= 0 ? d / cap : 0;
+    if (d < 0 || j >= P) {
+      ZB_FAIL(site, d, int64_t(P) * cap);
+      return nullptr;
+    }
     return reinterpret_cast<char*>(t.p[j]) + int64_t(d - j * cap) * row_bytes;
   }
 };
@@ -49,8 +57,10 @@ struct RankRows {
 // row addresses of token t (nullptr where d is out of range).
 template <int K, class T, class Rows>
 __device__ __forceinline__ void entry_rows(const Rows& rows, const int32_t* dst_row, int64_t t,
-                                           int64_t row_bytes, int lane, T* (&out)[K]) {
-  char* mine = lane < K ? rows.row(__ldg(dst_row + t * K + lane), row_bytes) : nullptr;
+                                           int64_t row_bytes, int lane, int site,
+                                           T* (&out)[K]) {
+  char* mine =
+      lane < K ? rows.row(__ldg(dst_row + t * K + lane), row_bytes, site) : nullptr;
 #pragma unroll
   for (int k = 0; k < K; ++k)
     out[k] = reinterpret_cast<T*>(
@@ -69,7 +79,7 @@ __global__ void __launch_bounds__(kMoveThreads) k_dispatch(int ntok, int H, Rows
   if (t >= ntok) return;
   const int nv = H >> 3;  // 16-byte vectors per row
   uint4* dst[K];
-  entry_rows<K>(rows, dst_row, t, int64_t(nv) * 16, lane, dst);  // out of range: skipped
+  entry_rows<K>(rows, dst_row, t, int64_t(nv) * 16, lane, ZB_SITE_DISPATCH_ROW, dst);
   const uint4* src = hidden + t * nv;
   for (int v0 = lane; v0 < nv; v0 += 32 * U) {
     uint4 x[U];
@@ -104,7 +114,7 @@ __global__ void __launch_bounds__(kMoveThreads) k_combine(int ntok, int H, Rows 
   if (t >= ntok) return;
   const int nv = H >> 3;
   const uint4* src[K];
-  entry_rows<K>(rows, dst_row, t, int64_t(nv) * 16, lane, src);
+  entry_rows<K>(rows, dst_row, t, int64_t(nv) * 16, lane, ZB_SITE_COMBINE_ROW, src);
   const float my_w = lane < K ? __ldg(w + t * K + lane) : 0.f;
   float wk[K];
   bool ok = true;
@@ -152,7 +162,7 @@ __global__ void __launch_bounds__(kMoveThreads) k_combine_wide(int ntok, int H, 
   if (t >= ntok) return;
   const int nv = H >> 4;  // 32-byte vectors per row
   const V8* src[K];
-  entry_rows<K>(rows, dst_row, t, int64_t(nv) * 32, lane, src);
+  entry_rows<K>(rows, dst_row, t, int64_t(nv) * 32, lane, ZB_SITE_COMBINE_ROW, src);
   const float my_w = lane < K ? __ldg(w + t * K + lane) : 0.f;
   float wk[K];
   bool ok = true;

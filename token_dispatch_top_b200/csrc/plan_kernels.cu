@@ -32,6 +32,7 @@
 #include "zb_internal.cuh"
 
 namespace zb {
+ZB_DEBUG_TU(debug_read_plan)
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
@@ -301,7 +302,7 @@ __device__ void greedy_warp(const PlanArgs& a, PlannerSmem& s, int T, int load, 
     int m = dload - T;
     m = min(m, T - rload);
     m = min(m, q);
-    if (lane == r) {
+    if (lane == r && ZB_IN(ZB_SITE_PLAN_SLOT, nfill, R)) {
       s.repe[r * R + nfill] = e;
       s.repq[r * R + nfill] = m;
       ++nfill;
@@ -625,7 +626,9 @@ __device__ long long emit_segments(const PlanArgs& a, const PlannerSmem& s, int 
             if (s.repe[j * R + r] == e) grp = Eh + r;
         }
         cum += inc - prev;
-        seg[idx++] = make_int2(cum, j * a.cap + s.cu[j * (G + 1) + grp] + prev);
+        if (ZB_IN(ZB_SITE_PLAN_SEGMENT, s.hoff[e] + idx, s.hoff[e + 1]))
+          seg[idx] = make_int2(cum, j * a.cap + s.cu[j * (G + 1) + grp] + prev);
+        ++idx;
       }
     }
   }
@@ -653,7 +656,7 @@ __device__ long long transport_warp(const PlanArgs& a, PlannerSmem& s, int e, in
       return 0;
     }
     const int inc = warp_incl_scan(d, lane);
-    if (lane < P)
+    if (lane < P && ZB_IN(ZB_SITE_PLAN_SEGMENT, s.hoff[e], s.hoff[e + 1]))
       seg[0] = make_int2(d, h0 * a.cap + s.cu[h0 * (G + 1) + (e - h0 * Eh)] + inc - d);
     return (long long)cost_a(lane, h0, gpn, a.inv_gpn) * d;
   }
@@ -778,7 +781,8 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
   __syncthreads();
   if (kMode == 2)
     for (int x = tid; x < P * R; x += kPlanThreads)
-      if (s.repe[x] >= 0) atomicOr(&s.hold[s.repe[x]], 1u << (x / R));
+      if (s.repe[x] >= 0 && ZB_IN(ZB_SITE_PLAN_SLOT, s.repe[x], E))
+        atomicOr(&s.hold[s.repe[x]], 1u << (x / R));
   __syncthreads();
 
   if (warp == 0) {
@@ -920,10 +924,11 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
       const int h0 = div_small(e, a.inv_eh);
       const int base = h0 * a.cap + s.cu[h0 * (G + 1) + (e - h0 * Eh)];
       const int h = s.hoff[e];
+      const bool in = ZB_IN(ZB_SITE_PLAN_SEGMENT, h, s.hoff[e + 1]);
       int run = 0;
       for (int i = 0; i < P; ++i) {
         const int d = s.cnt[i * E + e];
-        a.seg[int64_t(i) * a.seg_width + h] = make_int2(d, base + run);
+        if (in) a.seg[int64_t(i) * a.seg_width + h] = make_int2(d, base + run);
         cost_part += (long long)cost_a(i, h0, a.gpn, a.inv_gpn) * d;
         run += d;
       }
@@ -983,7 +988,7 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
   for (int u = 0; u < kPerThread; ++u) {
     const int t = w0 + 32 * u + lane;
     const int v = t < n ? __ldg(src + t) : -1;
-    ids[u] = unsigned(v) < unsigned(E) ? v : -1;
+    ids[u] = unsigned(v) < unsigned(E) && ZB_IN(ZB_SITE_ASSIGN_EXPERT, v, kMaxE) ? v : -1;
   }
   for (int x = tid; x < kAssignWarps * kMaxE; x += kChunkThreads) (&wh[0][0])[x] = 0;
   __syncthreads();
@@ -1036,6 +1041,7 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
     const int h_end = s_hoff[e + 1];
     int prev = 0, row = -1;
     for (int h = s_hoff[e]; h < h_end; ++h) {
+      if (!ZB_IN(ZB_SITE_ASSIGN_SEGMENT, h, a.seg_width)) break;
       const int2 sg = s_seg[h];
       if (p < sg.x) {
         row = sg.y + (p - prev);
@@ -1043,6 +1049,7 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
       }
       prev = sg.x;
     }
+    if (!ZB_IN(ZB_SITE_ASSIGN_ROW, row, nrows)) row = -1;
     const int64_t f = start + w0 + 32 * u + lane;
     a.dst_row[int64_t(il) * nk + f] = row;
     if (a.row_src && row >= 0 && int64_t(row) < nrows)
@@ -1117,7 +1124,8 @@ __global__ void __launch_bounds__(kEvalThreads) k_eval_placements(EvalArgs ea) {
   }
   __syncwarp();
   for (int x = lane; x < n; x += 32)
-    if (s.repe[x] >= 0) atomicOr(&s.hold[s.repe[x]], 1u << (x / R));
+    if (s.repe[x] >= 0 && ZB_IN(ZB_SITE_PLAN_SLOT, s.repe[x], E))
+      atomicOr(&s.hold[s.repe[x]], 1u << (x / R));
   __syncwarp();
   int L = 0;
   if (lane < P)

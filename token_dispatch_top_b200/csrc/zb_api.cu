@@ -317,4 +317,31 @@ int zb_combine(const zb_config* c, const zb_plan_t* plan, const uint16_t* y, con
   return ZB_OK;
 }
 
+int zb_debug_read(zb_debug_record* out, int reset) {
+#ifdef ZB_DEBUG
+  if (!out) return ZB_ERR_INVALID;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ZB_ERR_CUDA;
+  // the first failure reported is the first one recorded by the plan
+  // kernels, else by the data kernels, else by the merge kernels
+  cudaError_t (*const readers[])(zb::DebugRecord*, bool) = {
+      zb::debug_read_plan, zb::debug_read_move, zb::debug_read_merge};
+  *out = zb_debug_record{};
+  for (auto read : readers) {
+    zb::DebugRecord r{};
+    if (read(&r, reset != 0) != cudaSuccess) return ZB_ERR_CUDA;
+    if (r.count > 0 && out->count == 0) {
+      out->site = r.site;
+      out->index = r.index;
+      out->bound = r.bound;
+    }
+    out->count += r.count;
+  }
+  return ZB_OK;
+#else
+  (void)out;
+  (void)reset;
+  return ZB_ERR_INVALID;
+#endif
+}
+
 }  // extern "C"

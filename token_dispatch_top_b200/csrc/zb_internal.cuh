@@ -128,6 +128,54 @@ struct MergeArgs {
   int32_t* chunk_cnt;  // workspace [nchunk][P]
 };
 
+// Bounds checks.  ZB_IN(site, i, n) is 0 <= i < n for an access whose index
+// comes from data, and ZB_FAIL(site, i, n) marks a guard that has just
+// refused one.  In the release build ZB_IN is the constant true and ZB_FAIL
+// nothing, so both compile away (the guards that protect memory stay).  In
+// the debug build (ZB_DEBUG) a failure is counted, the first one's site,
+// index and bound are kept in the translation unit's device record, and the
+// access is skipped; zb_debug_read collects the records.  ZB_DEBUG_TU(name)
+// defines a translation unit's record and its host reader `name`.
+struct DebugRecord {
+  unsigned long long count;
+  long long index, bound;
+  int site, reserved;
+};
+
+#ifdef ZB_DEBUG
+#define ZB_DEBUG_TU(NAME)                                                          \
+  namespace {                                                                      \
+  __device__ DebugRecord g_debug;                                                  \
+  __device__ __noinline__ bool debug_fail(int site, long long i, long long n) {    \
+    if (atomicAdd(&g_debug.count, 1ull) == 0ull) {                                 \
+      g_debug.site = site;                                                         \
+      g_debug.index = i;                                                           \
+      g_debug.bound = n;                                                           \
+    }                                                                              \
+    return false;                                                                  \
+  }                                                                                \
+  }                                                                                \
+  cudaError_t NAME(DebugRecord* out, bool reset) {                                 \
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_debug, sizeof(DebugRecord));       \
+    if (e == cudaSuccess && reset) {                                               \
+      const DebugRecord zero{};                                                    \
+      e = cudaMemcpyToSymbol(g_debug, &zero, sizeof(DebugRecord));                 \
+    }                                                                              \
+    return e;                                                                      \
+  }
+#define ZB_IN(site, i, n)                                                   \
+  (((long long)(i) >= 0 && (long long)(i) < (long long)(n)) ||              \
+   debug_fail((site), (long long)(i), (long long)(n)))
+#define ZB_FAIL(site, i, n) ((void)debug_fail((site), (long long)(i), (long long)(n)))
+cudaError_t debug_read_plan(DebugRecord* out, bool reset);
+cudaError_t debug_read_move(DebugRecord* out, bool reset);
+cudaError_t debug_read_merge(DebugRecord* out, bool reset);
+#else
+#define ZB_DEBUG_TU(NAME)
+#define ZB_IN(site, i, n) true
+#define ZB_FAIL(site, i, n) ((void)0)
+#endif
+
 // Programmatic dependent launch.  A kernel launched with launch_pdl may start
 // while the kernel before it on the stream is still running, once every CTA
 // of that kernel has called griddep_launch_dependents (or exited).  Before

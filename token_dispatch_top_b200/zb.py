@@ -4,7 +4,8 @@ Every step of plan, dispatch and combine runs in the CUDA kernels of
 ``libzb.so``; this module passes ``torch.Tensor`` device pointers, sizes and
 the current CUDA stream to the C ABI declared in ``include/zb.h``.  There is
 no CPU fallback: if the library is missing or fails to load, every call
-raises.
+raises.  With ``ZB_DEBUG=1`` in the environment the bounds-checked build,
+``libzb_debug.so``, is loaded instead (see ``debug_read``).
 """
 from __future__ import annotations
 
@@ -17,7 +18,8 @@ import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libzb.so")
+DEBUG = os.environ.get("ZB_DEBUG", "") == "1"
+LIB_PATH = os.path.join(_HERE, "libzb_debug.so" if DEBUG else "libzb.so")
 
 OK = 0
 WARN_UNBALANCED = 1
@@ -39,7 +41,7 @@ EXPORTS = ("zb_strerror", "zb_validate", "zb_workspace_bytes", "zb_plan", "zb_pl
            "zb_merge", "zb_dispatch_merged", "zb_combine_reduce", "zb_combine_merged",
            "zb_recalibrate_workspace_bytes", "zb_recalibrate", "zb_place_by_demand",
            "zb_rank_workspace_bytes", "zb_count", "zb_plan_rank", "zb_dispatch_rank",
-           "zb_combine_rank")
+           "zb_combine_rank", "zb_debug_read")
 
 
 class ZbError(RuntimeError):
@@ -74,8 +76,9 @@ def load() -> ctypes.CDLL:
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise ImportError(f"libzb.so not built at {LIB_PATH}; run "
-                              "`python -m token_dispatch_top_b200.build`")
+            raise ImportError(f"{os.path.basename(LIB_PATH)} not built at {LIB_PATH}; run "
+                              "`python -m token_dispatch_top_b200.build"
+                              f"{' --debug' if LIB_PATH.endswith('_debug.so') else ''}`")
         lib = ctypes.CDLL(LIB_PATH)
         vp, cfgp, planp = ctypes.c_void_p, ctypes.POINTER(_Cfg), ctypes.POINTER(_Plan)
         lib.zb_strerror.argtypes = [ctypes.c_int]
@@ -108,12 +111,37 @@ def load() -> ctypes.CDLL:
                                      vp]
         lib.zb_dispatch_rank.argtypes = [cfgp, planp, vp, ctypes.POINTER(ctypes.c_void_p), vp]
         lib.zb_combine_rank.argtypes = [cfgp, planp, ctypes.POINTER(ctypes.c_void_p), vp, vp, vp]
+        lib.zb_debug_read.argtypes = [ctypes.POINTER(_DebugRecord), ctypes.c_int]
         _lib = lib
     return _lib
 
 
 def strerror(status: int) -> str:
     return load().zb_strerror(int(status)).decode()
+
+
+class _DebugRecord(ctypes.Structure):
+    _fields_ = [("count", ctypes.c_uint64), ("site", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("index", ctypes.c_int64),
+                ("bound", ctypes.c_int64)]
+
+
+# ZB_SITE_* of include/zb.h
+SITES = {1: "assign: expert id", 2: "assign: segment index", 3: "assign: row",
+         4: "planner: segment write", 5: "planner: slot or holder", 6: "dispatch: row",
+         7: "combine: row", 8: "merge: row"}
+
+
+def debug_read(reset: bool = True) -> dict:
+    """The bounds-checked build's record (synchronises the device): failed
+    checks since the last reset, and the site, index and bound of the first.
+    Raises in the release build, which keeps no record."""
+    rec = _DebugRecord()
+    st = load().zb_debug_read(ctypes.byref(rec), int(bool(reset)))
+    if st != OK:
+        raise ZbError(st, "zb_debug_read (the release library keeps no record)")
+    return {"count": int(rec.count), "site": SITES.get(int(rec.site), int(rec.site)),
+            "index": int(rec.index), "bound": int(rec.bound)}
 
 
 @dataclass(frozen=True)
