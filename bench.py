@@ -32,6 +32,9 @@ traffic.  Inputs are seeded and synthetic.
 * ``extras.workloads`` (N=1): the other four workloads one invocation at a
   time: plan latency, dispatch and combine rates and fractions of the peak,
   and the plan's balance (drift: steps 0, 31 and 63).
+* ``plan_timeline_us`` (N=1): per workload, the plan's device timeline from
+  its trace stamps: each kernel's start, release from its dependency wait
+  and end, in microseconds from the call's first kernel.
 * ``extras.rank_path`` (N=1): the entry points one rank of P GPUs calls
   (count, plan_rank, dispatch_rank, combine_rank) for each of the P ranks of
   the same workload in turn, each call timed alone; checked against the
@@ -305,6 +308,33 @@ def run_reference(args, wl, rank, budget_s: float = 120.0):
     print(json.dumps(line), flush=True)
 
 
+def plan_timeline(cfg, ids_list, dev, flush_l2, iters=10):
+    """The plan's device timeline from its trace (zb_plan_t.trace), each call
+    after an L2 flush and a device hold, on a plan object of its own (the
+    timed loops run untraced): per kernel, the median microseconds from the
+    call's first stamp to its first CTA's start, its release from its
+    dependency wait and its last CTA's end."""
+    import torch
+    from token_dispatch_top_b200 import zb
+    tplan = zb.Plan(cfg, dev, with_row_src=False, trace=True)
+    runs = []
+    for it in range(3 + iters):
+        flush_l2()
+        torch.cuda._sleep(SLEEP_CYCLES)
+        zb.plan(tplan, ids_list[it % len(ids_list)])
+        tl = zb.plan_trace(tplan)
+        if it >= 3:
+            runs.append(tl)
+    out = {}
+    for k in zb.TRACE_KERNELS:
+        if runs[0][k] is None:
+            out[k] = None
+            continue
+        out[k] = {f: statistics.median(r[k][f] for r in runs)
+                  for f in ("start", "released", "end")}
+    return out
+
+
 def measure_workload(wl, dev, flush_l2, peak, iters=10, steps=(0,)):
     """One workload's kernels, one invocation at a time (L2 flushed before
     each, outside the events): plan, dispatch and combine times, their HBM
@@ -363,6 +393,7 @@ def measure_workload(wl, dev, flush_l2, peak, iters=10, steps=(0,)):
                        "algorithmic_bytes": ab["combine"],
                        "kernel": "k_combine_wide (32-byte loads)"
                        if wl.K in (7, 8) and wl.H >= 4096 else "k_combine"},
+           "plan_timeline_us": plan_timeline(cfg, [x for x, _ in inputs], dev, flush_l2),
            "tokens_per_s": wl.tokens / ((pl + d + c) / 1000.0),
            "balance": balance}
     del plan, buf, out, hidden, inputs
@@ -804,6 +835,7 @@ def run_ours(args, wl, rank, world, local_rank):
     workloads = {}
     rank_path = None
     event_floor_us = None
+    timeline = None
     if world == 1 and args.extras:
         peak_gbs, _ = read_peaks()
         torch.cuda.empty_cache()
@@ -815,6 +847,7 @@ def run_ours(args, wl, rank, world, local_rank):
                                                steps=steps)
         # the per-rank entry points of the P-GPU form on this workload
         rank_path = measure_rank_path(wl, dev, flush_l2, peak_gbs)
+        timeline = plan_timeline(cfg, ids_l, dev, flush_l2)
         # what the same flush, hold and event pair read around the shortest
         # kernel there is (a one-element fill): the floor under every plan
         # latency above
@@ -922,6 +955,8 @@ def run_ours(args, wl, rank, world, local_rank):
                                "value": event_floor_us}},
         "plan_latency_us": dict({wl.name: 1000.0 * s_plan_ms / args.steps},
                                 **{k: v["plan_us"] for k, v in workloads.items()}),
+        "plan_timeline_us": dict({wl.name: timeline} if timeline else {},
+                                 **{k: v["plan_timeline_us"] for k, v in workloads.items()}),
         "wall_s": wall,
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,

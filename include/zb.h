@@ -142,7 +142,10 @@ typedef struct zb_config {
  *   dst_row     [P][S][K]     j*cap + row of each entry in the receive buffers
  *   row_src     [P][cap]      inverse of dst_row: g, or -1 for an unused row;
  *                             OPTIONAL, may be NULL (then not written)
- *   stats       int64 [ZB_STATS_LEN], see ZB_STAT_* */
+ *   stats       int64 [ZB_STATS_LEN], see ZB_STAT_*
+ *   trace       uint64 [ZB_TRACE_LEN]  device clock stamps of the plan's
+ *                             kernels, see ZB_TRACE_*; OPTIONAL, may be NULL
+ *                             (then not written) */
 typedef struct zb_plan_t {
   int32_t *cnt;
   int32_t *rep_expert;
@@ -154,7 +157,23 @@ typedef struct zb_plan_t {
   int32_t *dst_row;
   int32_t *row_src;
   int64_t *stats;
+  uint64_t *trace;
 } zb_plan_t;
+
+/* plan->trace, when not NULL: per kernel of the plan, three %globaltimer
+ * stamps (ns): the first of its CTAs to start, the first released by its
+ * wait on the kernel before it (k_zero has no wait: a second start stamp), and
+ * the last to finish.  The plan call resets them first (one more small
+ * launch on the stream); a kernel the call does not run (k_zero and k_hist
+ * in zb_plan_rank) keeps UINT64_MAX, UINT64_MAX, 0.  Kernels overlap under
+ * programmatic dependent launch, so a kernel may start before the one
+ * before it ends; its release stamp is when it could read that kernel's
+ * results. */
+#define ZB_TRACE_ZERO 0    /* k_zero: zeroes the per-source totals */
+#define ZB_TRACE_HIST 3    /* k_hist: histograms; waits on k_zero to add its totals */
+#define ZB_TRACE_PLANNER 6 /* k_planner: waits on k_hist */
+#define ZB_TRACE_ASSIGN 9  /* k_assign: waits on k_planner */
+#define ZB_TRACE_LEN 12
 
 /* Text of a status code (static storage; never NULL). */
 ZB_API const char *zb_strerror(int status);

@@ -118,6 +118,10 @@ def test_entry_points_reject_bad_arguments_without_a_device(lib):
         zb.ERR_INVALID
     assert lib.zb_plan(ctypes.byref(cfg), 16, ctypes.byref(fake), 128, ws, None) == \
         zb.ERR_INVALID
+    # a trace array that 64-bit atomics cannot use (not 8-byte aligned)
+    traced = zb._Plan(*([16] * 10), 12)
+    assert lib.zb_plan(ctypes.byref(cfg), 16, ctypes.byref(traced), 256, ws, None) == \
+        zb.ERR_INVALID
 
 
 def test_rank_entry_points_reject_bad_arguments_without_a_device(lib):

@@ -114,6 +114,30 @@ __device__ __forceinline__ int cost_a(int i, int j, int gpn, float inv_gpn) {
   return 1;
 }
 
+// Trace stamps (plan->trace): %globaltimer nanoseconds, the minimum over a
+// grid's CTAs for a start or a release from the dependency wait, the maximum
+// for an end.  Every stamp is skipped when the plan has no trace.
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void trace_first(const PlanArgs& a, int slot) {
+  if (a.trace != nullptr && threadIdx.x == 0) atomicMin(a.trace + slot, global_ns());
+}
+// Called by every thread of the CTA at the same point.
+__device__ __forceinline__ void trace_last(const PlanArgs& a, int slot) {
+  if (a.trace != nullptr) {
+    __syncthreads();
+    if (threadIdx.x == 0) atomicMax(a.trace + slot, global_ns());
+  }
+}
+
+__global__ void k_trace_reset(unsigned long long* trace) {
+  const int x = threadIdx.x;
+  if (x < ZB_TRACE_LEN) trace[x] = x % 3 == 2 ? 0ull : ~0ull;
+}
+
 // ------------------------------------------------------------------ step 1
 
 // One CTA per (chunk c, source rank i).  Thread t handles entries
@@ -123,6 +147,7 @@ __device__ __forceinline__ int cost_a(int i, int j, int gpn, float inv_gpn) {
 // slower, most of all on skewed batches (2.4 against 6.0 us on the hot one).
 __global__ void __launch_bounds__(kChunkThreads) k_hist(PlanArgs a) {
   __shared__ int32_t sh[kMaxE + 1];
+  trace_first(a, ZB_TRACE_HIST);
   griddep_launch_dependents();  // the planner may launch now and wait for us
   const int c = blockIdx.x, i = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
   const int E = a.E;
@@ -155,19 +180,24 @@ __global__ void __launch_bounds__(kChunkThreads) k_hist(PlanArgs a) {
   if (a.tot) {
     // the source's totals: zeroed by k_zero, this kernel's predecessor
     griddep_wait();
+    trace_first(a, ZB_TRACE_HIST + 1);
     int32_t* tot = a.tot + int64_t(i) * (E + 1);
     for (int e = tid; e <= E; e += kChunkThreads)
       if (sh[e]) atomicAdd(tot + e, sh[e]);
   }
+  trace_last(a, ZB_TRACE_HIST + 2);
 }
 
 // Zeroes the per-source totals k_hist adds into (the first kernel of a plan
 // on one GPU; k_hist, launched as its programmatic dependent, histograms its
 // chunk before waiting for it).
 __global__ void __launch_bounds__(kChunkThreads) k_zero(PlanArgs a, int n) {
+  trace_first(a, ZB_TRACE_ZERO);
+  trace_first(a, ZB_TRACE_ZERO + 1);
   griddep_launch_dependents();
   const int x = blockIdx.x * kChunkThreads + threadIdx.x;
   if (x < n) a.tot[x] = 0;
+  trace_last(a, ZB_TRACE_ZERO + 2);
 }
 
 // The count row of one source, counts[e] = sum over its chunks of
@@ -691,7 +721,9 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
   // the chunk histograms are read once k_hist has completed; from then on
   // the assignment CTAs may launch (they read their ids and the chunk
   // histograms before waiting for this plan)
+  trace_first(a, ZB_TRACE_PLANNER);
   griddep_wait();
+  trace_first(a, ZB_TRACE_PLANNER + 1);
   griddep_launch_dependents();
 
   // route counts cnt[i][e] (and ids outside [0, E)) summed over the chunks
@@ -760,6 +792,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
       for (int k = 0; k < ZB_STATS_LEN; ++k) a.stats[k] = 0;
       a.stats[ZB_STAT_STATUS] = ZB_ERR_INVALID;
     }
+    trace_last(a, ZB_TRACE_PLANNER + 2);
     return;
   }
   const int bad = s.misc[kMiscBad];
@@ -769,6 +802,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
       a.stats[ZB_STAT_STATUS] = ZB_ERR_BAD_ID;
       a.stats[ZB_STAT_BAD_IDS] = bad;
     }
+    trace_last(a, ZB_TRACE_PLANNER + 2);
     return;
   }
   // T_e, the initial home quotas, and the holders of each placed copy
@@ -954,6 +988,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
     a.stats[ZB_STAT_BAD_IDS] = 0;
     a.stats[ZB_STAT_REPAIRED] = s.misc[kMiscRepaired];
   }
+  trace_last(a, ZB_TRACE_PLANNER + 2);
 }
 
 // ------------------------------------------------------------------ step 3
@@ -972,6 +1007,7 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
   __shared__ int32_t wh[kAssignWarps][kMaxE];  // per-warp counts, then bases
   __shared__ int32_t s_hoff[kMaxE + 1];
   __shared__ int2 s_seg[kMaxSegWidth];
+  trace_first(a, ZB_TRACE_ASSIGN);
   const int c = blockIdx.x, il = blockIdx.y, i = a.src0 + il, tid = threadIdx.x,
             lane = tid & 31, warp = tid >> 5;
   const int E = a.E;
@@ -1024,13 +1060,17 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
     if (ids[u] >= 0) pos[u] += wh[warp][ids[u]];
 
   griddep_wait();  // the planner has completed: its tables are visible
+  trace_first(a, ZB_TRACE_ASSIGN + 1);
   // the plan's status and the tables this chunk reads, fetched together
   const int64_t status = a.stats[ZB_STAT_STATUS];
   for (int e = tid; e <= E; e += kChunkThreads) s_hoff[e] = a.hoff[e];
   const int2* segrow = a.seg + int64_t(i) * a.seg_width;
   for (int x = tid; x < a.seg_width; x += kChunkThreads) s_seg[x] = segrow[x];
   __syncthreads();
-  if (status < 0) return;  // bad ids or capacity: no rows
+  if (status < 0) {  // bad ids or capacity: no rows
+    trace_last(a, ZB_TRACE_ASSIGN + 2);
+    return;
+  }
   // pass 2: each entry's segment (the host its rank falls in) and row
   const int64_t nrows = int64_t(a.P) * a.cap;
 #pragma unroll
@@ -1055,6 +1095,7 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
     if (a.row_src && row >= 0 && int64_t(row) < nrows)
       a.row_src[row] = int32_t(int64_t(i) * nk + f);
   }
+  trace_last(a, ZB_TRACE_ASSIGN + 2);
 }
 
 // ------------------------------------------------ placement recalibration
@@ -1154,6 +1195,11 @@ size_t planner_smem_bytes(const zb_config& c) {
 cudaError_t launch_hist(const PlanArgs& a, int nsrc, cudaStream_t s) {
   if (a.nchunk == 0 || nsrc == 0) return cudaSuccess;
   k_hist<<<dim3(a.nchunk, nsrc), kChunkThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_trace_reset(unsigned long long* trace, cudaStream_t s) {
+  k_trace_reset<<<1, 32, 0, s>>>(trace);
   return cudaGetLastError();
 }
 

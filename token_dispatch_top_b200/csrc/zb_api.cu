@@ -23,6 +23,7 @@ int plan_buffers_ok(const zb_config& c, const zb_plan_t* p) {
     return 0;
   if (c.R > 0 && (!p->rep_expert || !p->rep_quota)) return 0;
   if (c.S > 0 && !p->dst_row) return 0;
+  if (reinterpret_cast<uintptr_t>(p->trace) & 7u) return 0;  // 64-bit atomics
   return 1;
 }
 
@@ -94,6 +95,7 @@ zb::PlanArgs plan_args(const zb_config* c, const zb::Workspace& w, const int32_t
     a.home_quota = plan->home_quota; a.load_before = plan->load_before;
     a.load_after = plan->load_after; a.cu_seqlens = plan->cu_seqlens;
     a.dst_row = plan->dst_row; a.row_src = plan->row_src; a.stats = plan->stats;
+    a.trace = reinterpret_cast<unsigned long long*>(plan->trace);
   }
   a.chunk_hist = reinterpret_cast<int32_t*>(base + w.off_chunk_hist);
   a.tot = nullptr;
@@ -124,6 +126,7 @@ int plan_impl(const zb_config* c, const int32_t* ids, const int32_t* placement,
   a.plan_hist = a.tot;
   a.plan_nchunk = 1;
 
+  if (a.trace && zb::launch_trace_reset(a.trace, s) != cudaSuccess) return ZB_ERR_CUDA;
   if (a.row_src &&
       cudaMemsetAsync(a.row_src, 0xff, sizeof(int32_t) * size_t(c->P) * c->cap_rows, s) !=
           cudaSuccess)
@@ -181,6 +184,7 @@ int zb_plan_rank(const zb_config* c, int rank, const int32_t* counts, const int3
   a.plan_hist = counts;
   a.plan_nchunk = 1;
   a.own_hist = a.chunk_hist;
+  if (a.trace && zb::launch_trace_reset(a.trace, s) != cudaSuccess) return ZB_ERR_CUDA;
   if (zb::launch_planner(a, zb::planner_smem_bytes(*c), s) != cudaSuccess) return ZB_ERR_CUDA;
   if (zb::launch_assign(a, 1, s) != cudaSuccess) return ZB_ERR_CUDA;
   return ZB_OK;

@@ -99,6 +99,7 @@ struct PlanArgs {
   int32_t* tot;  // [nsrc][E+1] per-source totals k_hist adds into, or nullptr
   int32_t* hoff;
   int2* seg;
+  unsigned long long* trace;  // plan->trace, or nullptr
 };
 
 // Candidate placements scored by the kept-placement greedy (recalibration).
@@ -206,6 +207,8 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 
 size_t planner_smem_bytes(const zb_config& c);
+
+cudaError_t launch_trace_reset(unsigned long long* trace, cudaStream_t s);
 
 cudaError_t launch_hist(const PlanArgs& a, int nsrc, cudaStream_t s);
 cudaError_t launch_hist_totals(const PlanArgs& a, int nsrc, cudaStream_t s);

@@ -35,6 +35,8 @@ POLICY_LOCAL = 1  # the largest move, then the most rows served locally
 STAT_STATUS, STAT_MAX_LOAD, STAT_N_REPLICAS, STAT_N_ITERS, STAT_WATER_LEVEL, \
     STAT_LOCALITY_COST, STAT_BAD_IDS, STAT_REPAIRED = range(8)
 STATS_LEN = 8
+TRACE_LEN = 12
+TRACE_KERNELS = ("k_zero", "k_hist", "k_planner", "k_assign")  # ZB_TRACE_* / 3
 
 EXPORTS = ("zb_strerror", "zb_validate", "zb_workspace_bytes", "zb_plan", "zb_plan_placed",
            "zb_plan_status", "zb_dispatch", "zb_combine", "zb_merge_workspace_bytes",
@@ -61,7 +63,7 @@ class _Cfg(ctypes.Structure):
 class _Plan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("cnt", "rep_expert", "rep_quota", "home_quota", "load_before", "load_after",
-                 "cu_seqlens", "dst_row", "row_src", "stats")]
+                 "cu_seqlens", "dst_row", "row_src", "stats", "trace")]
 
 
 class _Merge(ctypes.Structure):
@@ -118,6 +120,26 @@ def load() -> ctypes.CDLL:
 
 def strerror(status: int) -> str:
     return load().zb_strerror(int(status)).decode()
+
+
+def plan_trace(p) -> dict:
+    """The device timeline of the last plan call on ``p`` (a Plan or RankPlan
+    made with ``trace=True``; synchronises): per kernel, microseconds from the
+    first stamp of the call to the first of its CTAs to start, the first
+    released by its dependency wait, and the last to finish (None for a
+    kernel the call did not run)."""
+    if p.trace is None:
+        raise ZbError(ERR_INVALID, "plan_trace: the plan was made without trace=True")
+    t = p.trace.cpu().numpy().view(np.uint64)
+    never = np.uint64(0xFFFFFFFFFFFFFFFF)
+    t0 = min(int(t[3 * k]) for k in range(len(TRACE_KERNELS)) if t[3 * k] != never)
+    out = {}
+    for k, name in enumerate(TRACE_KERNELS):
+        st, rel, en = (int(x) for x in t[3 * k:3 * k + 3])
+        out[name] = None if t[3 * k] == never else {
+            "start": (st - t0) / 1000.0, "released": (rel - t0) / 1000.0,
+            "end": (en - t0) / 1000.0}
+    return out
 
 
 class _DebugRecord(ctypes.Structure):
@@ -190,7 +212,7 @@ def workspace_bytes(cfg: Config) -> int:
 class Plan:
     """Device buffers of one plan plus its scratch workspace (torch-owned)."""
 
-    def __init__(self, cfg: Config, device, with_row_src: bool = True):
+    def __init__(self, cfg: Config, device, with_row_src: bool = True, trace: bool = False):
         if validate(cfg) != OK:
             raise ZbError(ERR_INVALID, f"config {cfg}")
         i32 = dict(dtype=torch.int32, device=device)
@@ -206,6 +228,8 @@ class Plan:
         self.dst_row = torch.empty((P, cfg.S, cfg.K), **i32)
         self.row_src = torch.empty((P, cfg.cap), **i32) if with_row_src else None
         self.stats = torch.zeros((STATS_LEN,), dtype=torch.int64, device=device)
+        self.trace = torch.zeros((TRACE_LEN,), dtype=torch.int64, device=device) \
+            if trace else None
         self.ws_bytes = workspace_bytes(cfg)
         self.workspace = torch.empty((self.ws_bytes + 256,), dtype=torch.uint8, device=device)
         self.ws_ptr = (self.workspace.data_ptr() + 255) & ~255  # 256-byte aligned
@@ -215,7 +239,7 @@ class Plan:
             return None if t is None or t.numel() == 0 else t.data_ptr()
         self._p = _Plan(p(self.cnt), p(self.rep_expert), p(self.rep_quota), p(self.home_quota),
                         p(self.load_before), p(self.load_after), p(self.cu_seqlens),
-                        p(self.dst_row), p(self.row_src), p(self.stats))
+                        p(self.dst_row), p(self.row_src), p(self.stats), p(self.trace))
 
 
 def _stream(stream) -> int:
@@ -406,7 +430,7 @@ class RankPlan:
     count row ``counts`` [E+1], the all-gathered table ``table`` [P,E+1] and
     the scratch workspace that ``count`` fills and ``plan_rank`` reads."""
 
-    def __init__(self, cfg: Config, rank: int, device):
+    def __init__(self, cfg: Config, rank: int, device, trace: bool = False):
         if validate(cfg) != OK or not 0 <= rank < cfg.P:
             raise ZbError(ERR_INVALID, f"config {cfg}, rank {rank}")
         i32 = dict(dtype=torch.int32, device=device)
@@ -421,6 +445,8 @@ class RankPlan:
         self.cu_seqlens = torch.empty((P, cfg.Eh + R + 1), **i32)
         self.dst_row = torch.empty((cfg.S, cfg.K), **i32)
         self.stats = torch.zeros((STATS_LEN,), dtype=torch.int64, device=device)
+        self.trace = torch.zeros((TRACE_LEN,), dtype=torch.int64, device=device) \
+            if trace else None
         self.counts = torch.empty((E + 1,), **i32)
         self.table = torch.empty((P, E + 1), **i32)
         self.ws_bytes = int(load().zb_rank_workspace_bytes(ctypes.byref(cfg.c())))
@@ -432,7 +458,7 @@ class RankPlan:
             return None if t is None or t.numel() == 0 else t.data_ptr()
         self._p = _Plan(p(self.cnt), p(self.rep_expert), p(self.rep_quota), p(self.home_quota),
                         p(self.load_before), p(self.load_after), p(self.cu_seqlens),
-                        p(self.dst_row), None, p(self.stats))
+                        p(self.dst_row), None, p(self.stats), p(self.trace))
 
 
 def count(rp: RankPlan, topk_ids: torch.Tensor, stream=None) -> None:
