@@ -367,6 +367,23 @@ def test_bad_ids_write_nothing(dev):
     assert bool((out.view(torch.int16) == parity.SENTINEL).all())
 
 
+@pytest.mark.parametrize("P,E,K,S", [(8, 32, 2, 39000), (4, 16, 8, 298000)])
+def test_assign_several_chunks_per_cta(dev, P, E, K, S):
+    """Batches whose assignment grid would not fit the device at once, so each
+    assignment CTA takes 2 (P=8: 39 chunks per source) or 4 consecutive chunks
+    (P=4: 1165 chunks per source), the last CTA fewer, the last chunk ragged:
+    the whole plan, dst_row and row_src bit-exact."""
+    rng = np.random.default_rng(P)
+    pop = 1.0 / np.arange(1, E + 1) ** 1.1
+    ids = rng.choice(E, size=(P, S, K), p=pop[rng.permutation(E)] / pop.sum()).astype(np.int32)
+    kw = dict(P=P, E=E, K=K, S=S, H=8, R=2, C=0.0, cap_rows=2 * S * K)
+    zc, oc = zb.Config(**kw), oracle.Config(**kw)
+    p, status, _ = gpu_plan(zc, ids, dev)
+    assert_plan_equal(plan_tables(p), oracle.plan(oc, ids, want_M=False), status)
+    del p
+    torch.cuda.empty_cache()
+
+
 def test_ids_far_out_of_range(dev):
     """Ids far outside [0, E) (beyond every table an id indexes) are counted
     and stop the plan like any bad id; the same on the per-rank entry points.

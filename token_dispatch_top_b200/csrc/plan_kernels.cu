@@ -28,6 +28,7 @@
 // enforces and how" (S x K per rank, cu_seqlens, expert-grouped fixed
 // buffers).
 #include <atomic>
+#include <mutex>
 
 #include "zb_internal.cuh"
 
@@ -996,72 +997,90 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
 constexpr int kAssignWarps = kChunkThreads / 32;
 constexpr int kPerWarp = kChunk / kAssignWarps;  // kPerThread steps of 32
 
-// One CTA per (chunk c, source rank i).  Warp w owns entries
-// [kPerWarp*w, kPerWarp*(w+1)) of the chunk and walks them 32 at a time in flat
-// order, so ranks among equal experts come out in flat-index order.  Each
-// entry's rank within the source's entries of its expert (earlier chunks,
-// earlier warps, the warp's earlier slices, lower lanes) depends on nothing
-// the planner writes, so it is complete before the wait; after it only the
-// segment lookup and the stores remain.
-__global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
+// One CTA per (a.assign_sub consecutive chunks, source rank i).  The host
+// gives a CTA several chunks when one per CTA would not fit on the device at
+// once, so that every CTA does its share of the work below while the planner
+// runs.  Within a chunk, warp w owns entries [kPerWarp*w, kPerWarp*(w+1)) and
+// walks them 32 at a time in flat order, so ranks among equal experts come
+// out in flat-index order.  Each entry's rank within the source's entries of
+// its expert (earlier chunks, earlier warps, the warp's earlier slices,
+// lower lanes) depends on nothing the planner writes, so it is complete
+// before the wait, and staged in shared memory with the entry's expert;
+// after the wait only the segment lookup and the stores remain.
+__global__ void __launch_bounds__(kChunkThreads, 2) k_assign(PlanArgs a) {
   __shared__ int32_t wh[kAssignWarps][kMaxE];  // per-warp counts, then bases
+  __shared__ int32_t s_run[kMaxE];             // prefix of the chunks before
   __shared__ int32_t s_hoff[kMaxE + 1];
   __shared__ int2 s_seg[kMaxSegWidth];
+  extern __shared__ int32_t s_ent[];  // per chunk: kChunk experts, kChunk ranks
   trace_first(a, ZB_TRACE_ASSIGN);
-  const int c = blockIdx.x, il = blockIdx.y, i = a.src0 + il, tid = threadIdx.x,
-            lane = tid & 31, warp = tid >> 5;
+  const int nsub = a.assign_sub, c0 = blockIdx.x * nsub, il = blockIdx.y, i = a.src0 + il,
+            tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int E = a.E;
   const int64_t nk = int64_t(a.S) * a.K;
-  const int64_t start = int64_t(c) * kChunk;
-  const int n = (nk - start) < kChunk ? int(nk - start) : kChunk;
-  const int32_t* src = a.ids + int64_t(il) * nk + start;
   const int w0 = warp * kPerWarp;
-  // ids outside [0, E) become -1 here: they are counted by k_hist and stop
-  // the plan (ZB_ERR_BAD_ID) before any row is written, and no table below
-  // is indexed by them
-  int ids[kPerThread];
-#pragma unroll
-  for (int u = 0; u < kPerThread; ++u) {
-    const int t = w0 + 32 * u + lane;
-    const int v = t < n ? __ldg(src + t) : -1;
-    ids[u] = unsigned(v) < unsigned(E) && ZB_IN(ZB_SITE_ASSIGN_EXPERT, v, kMaxE) ? v : -1;
-  }
-  for (int x = tid; x < kAssignWarps * kMaxE; x += kChunkThreads) (&wh[0][0])[x] = 0;
-  __syncthreads();
+  const int32_t* hist = a.chunk_hist + int64_t(il) * a.nchunk * (E + 1);
 
-  // pass 1: each entry's rank among the warp's entries of its expert so far,
-  // and the per-warp histogram
-  int pos[kPerThread];
+  for (int sub = 0; sub < nsub && c0 + sub < a.nchunk; ++sub) {
+    const int c = c0 + sub;
+    const int64_t start = int64_t(c) * kChunk;
+    const int n = (nk - start) < kChunk ? int(nk - start) : kChunk;
+    const int32_t* src = a.ids + int64_t(il) * nk + start;
+    // ids outside [0, E) become -1 here: they are counted by k_hist and stop
+    // the plan (ZB_ERR_BAD_ID) before any row is written, and no table below
+    // is indexed by them
+    int ids[kPerThread];
 #pragma unroll
-  for (int u = 0; u < kPerThread; ++u) {
-    const int e = ids[u];
-    const unsigned peers = __match_any_sync(kFull, e);
-    pos[u] = e >= 0 ? wh[warp][e] + __popc(peers & ((1u << lane) - 1u)) : 0;
-    __syncwarp();
-    if (e >= 0 && lane == __ffs(peers) - 1) wh[warp][e] += __popc(peers);
-    __syncwarp();
-  }
-  __syncthreads();
-  // exclusive prefix: earlier chunks of this source, then earlier warps.  The
-  // chunk histograms are complete: the planner launches this kernel only
-  // after its own wait on k_hist has returned.
-  for (int e = tid; e < E; e += kChunkThreads) {
-    int run = strided_sum<16>(a.chunk_hist + int64_t(il) * a.nchunk * (E + 1) + e, c, E + 1);
-#pragma unroll
-    for (int w = 0; w < kAssignWarps; ++w) {
-      const int v = wh[w][e];
-      wh[w][e] = run;
-      run += v;
+    for (int u = 0; u < kPerThread; ++u) {
+      const int t = w0 + 32 * u + lane;
+      const int v = t < n ? __ldg(src + t) : -1;
+      ids[u] = unsigned(v) < unsigned(E) && ZB_IN(ZB_SITE_ASSIGN_EXPERT, v, kMaxE) ? v : -1;
     }
-  }
-  __syncthreads();
+    for (int x = tid; x < kAssignWarps * kMaxE; x += kChunkThreads) (&wh[0][0])[x] = 0;
+    __syncthreads();
+
+    // pass 1: each entry's rank among the warp's entries of its expert so
+    // far, and the per-warp histogram
+    int pos[kPerThread];
 #pragma unroll
-  for (int u = 0; u < kPerThread; ++u)
-    if (ids[u] >= 0) pos[u] += wh[warp][ids[u]];
+    for (int u = 0; u < kPerThread; ++u) {
+      const int e = ids[u];
+      const unsigned peers = __match_any_sync(kFull, e);
+      pos[u] = e >= 0 ? wh[warp][e] + __popc(peers & ((1u << lane) - 1u)) : 0;
+      __syncwarp();
+      if (e >= 0 && lane == __ffs(peers) - 1) wh[warp][e] += __popc(peers);
+      __syncwarp();
+    }
+    __syncthreads();
+    // exclusive prefix: earlier chunks of this source, then earlier warps.
+    // The chunk histograms are complete: the planner launches this kernel
+    // only after its own wait on k_hist has returned.  The first chunk of
+    // the CTA sums the chunk histograms before it; each next one adds the
+    // chunk just done.
+    for (int e = tid; e < E; e += kChunkThreads) {
+      int run = sub == 0 ? strided_sum<16>(hist + e, c, E + 1) : s_run[e];
+#pragma unroll
+      for (int w = 0; w < kAssignWarps; ++w) {
+        const int v = wh[w][e];
+        wh[w][e] = run;
+        run += v;
+      }
+      s_run[e] = run;
+    }
+    __syncthreads();
+    int32_t* ent = s_ent + sub * 2 * kChunk;
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+      const int t = w0 + 32 * u + lane;
+      ent[t] = ids[u];
+      ent[kChunk + t] = ids[u] >= 0 ? pos[u] + wh[warp][ids[u]] : 0;
+    }
+    __syncthreads();  // wh is zeroed again for the next chunk
+  }
 
   griddep_wait();  // the planner has completed: its tables are visible
   trace_first(a, ZB_TRACE_ASSIGN + 1);
-  // the plan's status and the tables this chunk reads, fetched together
+  // the plan's status and the tables this CTA reads, fetched together
   const int64_t status = a.stats[ZB_STAT_STATUS];
   for (int e = tid; e <= E; e += kChunkThreads) s_hoff[e] = a.hoff[e];
   const int2* segrow = a.seg + int64_t(i) * a.seg_width;
@@ -1073,27 +1092,32 @@ __global__ void __launch_bounds__(kChunkThreads) k_assign(PlanArgs a) {
   }
   // pass 2: each entry's segment (the host its rank falls in) and row
   const int64_t nrows = int64_t(a.P) * a.cap;
+  for (int sub = 0; sub < nsub && c0 + sub < a.nchunk; ++sub) {
+    const int64_t start = int64_t(c0 + sub) * kChunk;
+    const int32_t* ent = s_ent + sub * 2 * kChunk;
 #pragma unroll
-  for (int u = 0; u < kPerThread; ++u) {
-    const int e = ids[u];
-    if (e < 0) continue;
-    const int p = pos[u];
-    const int h_end = s_hoff[e + 1];
-    int prev = 0, row = -1;
-    for (int h = s_hoff[e]; h < h_end; ++h) {
-      if (!ZB_IN(ZB_SITE_ASSIGN_SEGMENT, h, a.seg_width)) break;
-      const int2 sg = s_seg[h];
-      if (p < sg.x) {
-        row = sg.y + (p - prev);
-        break;
+    for (int u = 0; u < kPerThread; ++u) {
+      const int t = w0 + 32 * u + lane;
+      const int e = ent[t];
+      if (e < 0) continue;
+      const int p = ent[kChunk + t];
+      const int h_end = s_hoff[e + 1];
+      int prev = 0, row = -1;
+      for (int h = s_hoff[e]; h < h_end; ++h) {
+        if (!ZB_IN(ZB_SITE_ASSIGN_SEGMENT, h, a.seg_width)) break;
+        const int2 sg = s_seg[h];
+        if (p < sg.x) {
+          row = sg.y + (p - prev);
+          break;
+        }
+        prev = sg.x;
       }
-      prev = sg.x;
+      if (!ZB_IN(ZB_SITE_ASSIGN_ROW, row, nrows)) row = -1;
+      const int64_t f = start + t;
+      a.dst_row[int64_t(il) * nk + f] = row;
+      if (a.row_src && row >= 0 && int64_t(row) < nrows)
+        a.row_src[row] = int32_t(int64_t(i) * nk + f);
     }
-    if (!ZB_IN(ZB_SITE_ASSIGN_ROW, row, nrows)) row = -1;
-    const int64_t f = start + w0 + 32 * u + lane;
-    a.dst_row[int64_t(il) * nk + f] = row;
-    if (a.row_src && row >= 0 && int64_t(row) < nrows)
-      a.row_src[row] = int32_t(int64_t(i) * nk + f);
   }
   trace_last(a, ZB_TRACE_ASSIGN + 2);
 }
@@ -1271,9 +1295,49 @@ cudaError_t launch_eval_placements(const EvalArgs& ea, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// Chunks per assignment CTA: the fewest (at most kMaxAssignSub) with which
+// every CTA of the grid fits on the device at once, beside the planner's CTA,
+// from the occupancy of k_assign at each staging size (computed once per
+// device).
+int assign_sub(int nchunk, int nsrc) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static int resident[kMaxDevices][kMaxAssignSub + 1];
+  static bool known[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  int local[kMaxAssignSub + 1] = {};
+  int* res = dev < kMaxDevices ? resident[dev] : local;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= kMaxDevices || !known[dev]) {
+      int sms = 0;
+      if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+          cudaFuncSetAttribute(k_assign, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               int(assign_smem_bytes(kMaxAssignSub))) != cudaSuccess)
+        return 1;
+      for (int sub = 1; sub <= kMaxAssignSub; ++sub) {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_assign, kChunkThreads,
+                                                          assign_smem_bytes(sub)) !=
+            cudaSuccess)
+          return 1;
+        res[sub] = per_sm * (sms - 1);  // the planner's CTA holds one SM meanwhile
+      }
+      if (dev < kMaxDevices) known[dev] = true;
+    }
+  }
+  for (int sub = 1; sub <= kMaxAssignSub; ++sub)
+    if (ceil_div(nchunk, sub) * nsrc <= res[sub]) return sub;
+  return kMaxAssignSub;
+}
+
 cudaError_t launch_assign(const PlanArgs& a, int nsrc, cudaStream_t s) {
   if (a.nchunk == 0 || nsrc == 0) return cudaSuccess;
-  return launch_pdl(k_assign, dim3(a.nchunk, nsrc), dim3(kChunkThreads), 0, s, a);
+  PlanArgs b = a;
+  b.assign_sub = assign_sub(a.nchunk, nsrc);
+  return launch_pdl(k_assign, dim3(unsigned(ceil_div(a.nchunk, b.assign_sub)), nsrc),
+                    dim3(kChunkThreads), assign_smem_bytes(b.assign_sub), s, b);
 }
 
 }  // namespace zb

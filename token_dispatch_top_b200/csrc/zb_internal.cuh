@@ -100,7 +100,12 @@ struct PlanArgs {
   int32_t* hoff;
   int2* seg;
   unsigned long long* trace;  // plan->trace, or nullptr
+  int assign_sub;             // chunks per k_assign CTA (set by launch_assign)
 };
+
+// k_assign stages each of its chunks' experts and ranks in shared memory.
+constexpr int kMaxAssignSub = 4;
+inline size_t assign_smem_bytes(int sub) { return size_t(sub) * 2 * kChunk * sizeof(int32_t); }
 
 // Candidate placements scored by the kept-placement greedy (recalibration).
 constexpr int kEvalThreads = 256;
