@@ -69,36 +69,6 @@ __device__ __forceinline__ int strided_sum(const int32_t* col, int n, int64_t st
   return v;
 }
 
-// Column sums of a [rows][nchunk][ncol_row] table for the four columns
-// x0 + u*step (u < 4) of the flattened [rows][ncol_row] index space below
-// ncol: v[u] = sum over c of table[row][c][col].  Thirty-two loads in flight
-// per thread.
-__device__ __forceinline__ void column_sums4(const int32_t* table, int nchunk, int ncol_row,
-                                             int ncol, int x0, int step, int (&v)[4]) {
-  const int32_t* col[4];
-  bool ok[4];
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int x = x0 + u * step;
-    ok[u] = x < ncol;
-    const int i = ok[u] ? x / ncol_row : 0, e = ok[u] ? x - i * ncol_row : 0;
-    col[u] = table + int64_t(i) * nchunk * ncol_row + e;
-    v[u] = 0;
-  }
-  for (int c = 0; c < nchunk; c += 8) {
-    int t[4][8];
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        t[u][k] = (ok[u] && c + k < nchunk) ? col[u][int64_t(c + k) * ncol_row] : 0;
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-#pragma unroll
-      for (int k = 0; k < 8; ++k) v[u] += t[u][k];
-  }
-}
-
 // r / g for the planner's small non-negative integers (ranks, experts), from
 // inv = float(1/g): (r + 1/2) / g lies at least 1/(2g) from an integer, and
 // for r < 2^22 the float product (r + 1/2) * inv is within (r + 1/2) / g *
@@ -716,6 +686,7 @@ template <int kMode, bool kRepair, bool kBand>
 __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
   extern __shared__ __align__(16) char smem_raw[];
   __shared__ unsigned long long s_cost;
+  __shared__ int s_wsum[3][kPlanWarps];  // per warp of experts: hosts, replicated, home-only
   PlannerSmem s = carve(smem_raw, a);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int P = a.P, E = a.E, R = a.R, Eh = a.Eh, G = Eh + R;
@@ -727,7 +698,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
   trace_first(a, ZB_TRACE_PLANNER + 1);
   griddep_launch_dependents();
 
-  // route counts cnt[i][e] (and ids outside [0, E)) summed over the chunks
+  // route counts cnt[i][e] and ids outside [0, E), one row per source
   if (tid == 0) {
     s.misc[kMiscBad] = 0;
     s.misc[kMiscErr] = 0;
@@ -736,12 +707,15 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
     s_cost = 0ull;
   }
   __syncthreads();
-  // (four columns per thread at a time, eight chunks of each in flight)
-  for (int x0 = tid; x0 < P * (E + 1); x0 += 4 * kPlanThreads) {
-    int v[4];
-    column_sums4(a.plan_hist, a.plan_nchunk, E + 1, P * (E + 1), x0, kPlanThreads, v);
+  for (int x0 = tid; x0 < P * (E + 1); x0 += 8 * kPlanThreads) {
+    int v[8];  // eight columns of the table per thread in flight
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 8; ++u) {
+      const int x = x0 + u * kPlanThreads;
+      v[u] = x < P * (E + 1) ? __ldcg(a.plan_hist + x) : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
       const int x = x0 + u * kPlanThreads;
       if (x >= P * (E + 1)) break;
       const int i = x / (E + 1), e = x - i * (E + 1);
@@ -867,30 +841,46 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
     a.rep_expert[x] = s.repe[x];
     a.rep_quota[x] = s.repq[x];
   }
-  // hosts per expert and their first segment index (one warp scans E)
-  if (warp == 0) {
-    int carry = 0;
-    for (int e0 = 0; e0 < E; e0 += 32) {
-      const int e = e0 + lane;
-      const int nh = e < E ? 1 + __popc(s.hold[e]) : 0;
-      const int inc = warp_incl_scan(nh, lane);
-      if (e < E) s.hoff[e] = carry + inc - nh;
-      carry += __shfl_sync(kFull, inc, 31);
+  // hosts per expert and their first segment index, and the transport
+  // order: experts with replicas (the long case) first, so that they land on
+  // different warps, then the experts served by home alone, each by expert
+  // id.  Warp w scans experts [32w, 32w + 32) (E <= kMaxE = 12 warps of
+  // them), then adds the totals of the warps before it.
+  static_assert(kMaxE <= 32 * kPlanWarps, "one warp per 32 experts");
+  const int nwe = (E + 31) / 32;
+  const int e_mine = warp * 32 + lane;
+  const bool e_in = warp < nwe && e_mine < E;
+  const int nh = e_in ? 1 + __popc(s.hold[e_mine]) : 0;
+  const bool rep = nh > 1;
+  int nh_inc = 0;
+  unsigned m_rep = 0u, m_home = 0u;
+  if (warp < nwe) {
+    nh_inc = warp_incl_scan(nh, lane);
+    m_rep = __ballot_sync(kFull, rep);
+    m_home = __ballot_sync(kFull, e_in && !rep);
+    if (lane == 31) s_wsum[0][warp] = nh_inc;
+    if (lane == 0) {
+      s_wsum[1][warp] = __popc(m_rep);
+      s_wsum[2][warp] = __popc(m_home);
     }
-    if (lane == 0) s.hoff[E] = carry;
-    // transport order: experts with replicas (the long case) first, so that
-    // they land on different warps, then the experts served by home alone
-    int n = 0;
-    for (int pass = 0; pass < 2; ++pass) {
-      for (int e0 = 0; e0 < E; e0 += 32) {
-        const int e = e0 + lane;
-        const bool take = e < E && ((s.hold[e] != 0u) == (pass == 0));
-        const unsigned m = __ballot_sync(kFull, take);
-        if (take) s.order[n + __popc(m & ((1u << lane) - 1u))] = e;
-        n += __popc(m);
+  }
+  __syncthreads();
+  if (warp < nwe) {
+    int off_h = 0, off_r = 0, off_o = 0, nrx = 0;
+    for (int w = 0; w < nwe; ++w) {
+      if (w < warp) {
+        off_h += s_wsum[0][w];
+        off_r += s_wsum[1][w];
+        off_o += s_wsum[2][w];
       }
-      if (pass == 0 && lane == 0) s.misc[kMiscNRepExp] = n;
+      nrx += s_wsum[1][w];
     }
+    if (e_in) s.hoff[e_mine] = off_h + nh_inc - nh;
+    if (warp == nwe - 1 && lane == 31) s.hoff[E] = off_h + nh_inc;
+    const unsigned below = (1u << lane) - 1u;
+    if (rep) s.order[off_r + __popc(m_rep & below)] = e_mine;
+    if (e_in && !rep) s.order[nrx + off_o + __popc(m_home & below)] = e_mine;
+    if (warp == 0 && lane == 0) s.misc[kMiscNRepExp] = nrx;
   }
   int32_t* Mw = s.M + warp * 32 * 32;
   int32_t* qw = s.q + warp * 32;

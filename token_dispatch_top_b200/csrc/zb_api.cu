@@ -102,8 +102,7 @@ zb::PlanArgs plan_args(const zb_config* c, const zb::Workspace& w, const int32_t
   a.hoff = reinterpret_cast<int32_t*>(base + w.off_hoff);
   a.seg = reinterpret_cast<int2*>(base + w.off_seg);
   a.src0 = 0;
-  a.plan_hist = a.chunk_hist;
-  a.plan_nchunk = w.nchunk;
+  a.plan_hist = nullptr;  // set by the calls that plan
   a.own_hist = nullptr;
   return a;
 }
@@ -124,7 +123,6 @@ int plan_impl(const zb_config* c, const int32_t* ids, const int32_t* placement,
   // the planner reads the per-source totals that k_hist adds up
   a.tot = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + w.off_tot);
   a.plan_hist = a.tot;
-  a.plan_nchunk = 1;
 
   if (a.trace && zb::launch_trace_reset(a.trace, s) != cudaSuccess) return ZB_ERR_CUDA;
   if (a.row_src &&
@@ -182,7 +180,6 @@ int zb_plan_rank(const zb_config* c, int rank, const int32_t* counts, const int3
   zb::PlanArgs a = plan_args(c, w, ids, c->R > 0 ? placement : nullptr, plan, ws);
   a.src0 = rank;
   a.plan_hist = counts;
-  a.plan_nchunk = 1;
   a.own_hist = a.chunk_hist;
   if (a.trace && zb::launch_trace_reset(a.trace, s) != cudaSuccess) return ZB_ERR_CUDA;
   if (zb::launch_planner(a, zb::planner_smem_bytes(*c), s) != cudaSuccess) return ZB_ERR_CUDA;

@@ -65,10 +65,9 @@ inline Workspace workspace_layout(const zb_config& c, int nsrc) {
 
 // Kernel parameter block shared by the plan kernels.
 //
-// The planner reads the route counts from plan_hist [P][plan_nchunk][E+1],
-// summing each column over its chunks: the per-source totals k_hist adds up
-// (whole batch on one GPU), or the exchanged count rows of P ranks (both
-// with plan_nchunk = 1).  k_hist and k_assign handle the sources src0 ..
+// The planner reads the route counts from plan_hist [P][E+1]: the
+// per-source totals k_hist adds up (whole batch on one GPU), or the exchanged
+// count rows of P ranks.  k_hist and k_assign handle the sources src0 ..
 // src0 + gridDim.y - 1; ids, dst_row and chunk_hist are indexed from src0
 // (local), seg and row_src by the global source.  own_hist, when set, holds
 // the per-chunk histograms of source src0 alone, which the planner checks
@@ -80,7 +79,6 @@ struct PlanArgs {
   int nchunk, seg_width;
   float inv_gpn, inv_eh;  // 1/gpn and 1/Eh, for div_small
   int src0;
-  int plan_nchunk;
   const int32_t* plan_hist;
   const int32_t* own_hist;
   const int32_t* ids;
