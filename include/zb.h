@@ -184,8 +184,9 @@ ZB_API int zb_validate(const zb_config *cfg);
 
 /* Bytes of device scratch memory zb_plan needs for `cfg` (0 if `cfg` is
  * invalid).  Host only.  The workspace holds the per-chunk histograms, the
- * per-(source, expert) segment table and error flags; its contents need not
- * be initialised and are dead after the plan's kernels complete. */
+ * per-source totals, the first segment of each expert and the per-(source,
+ * expert) segment table; its contents need not be initialised and are dead
+ * after the plan's kernels complete. */
 ZB_API size_t zb_workspace_bytes(const zb_config *cfg);
 
 /* Steps 1-3: histogram, greedy replica plan, assignment.
@@ -221,7 +222,8 @@ ZB_API size_t zb_workspace_bytes(const zb_config *cfg);
  * zb_plan_t.  workspace: device, zb_workspace_bytes(cfg) bytes (pass that
  * count as workspace_bytes), 256-byte aligned.
  * Returns ZB_OK once the work is enqueued, ZB_ERR_INVALID (bad cfg, NULL
- * buffer, short workspace) or ZB_ERR_CUDA.  The plan's own outcome (OK,
+ * buffer, short or misaligned workspace, a trace array not 8-byte aligned)
+ * or ZB_ERR_CUDA.  The plan's own outcome (OK,
  * UNBALANCED, CAPACITY, BAD_ID) lands in plan->stats; read it with
  * zb_plan_status.  On CAPACITY or BAD_ID, dst_row and row_src are undefined. */
 ZB_API int zb_plan(const zb_config *cfg, const int32_t *topk_ids, const zb_plan_t *plan,
