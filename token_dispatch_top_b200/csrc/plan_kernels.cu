@@ -707,6 +707,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
     s_cost = 0ull;
   }
   __syncthreads();
+  const float inv_e1 = 1.0f / float(E + 1);  // for div_small: x < 32 * 385 < 2^22
   for (int x0 = tid; x0 < P * (E + 1); x0 += 8 * kPlanThreads) {
     int v[8];  // eight columns of the table per thread in flight
 #pragma unroll
@@ -718,7 +719,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_planner(PlanArgs a) {
     for (int u = 0; u < 8; ++u) {
       const int x = x0 + u * kPlanThreads;
       if (x >= P * (E + 1)) break;
-      const int i = x / (E + 1), e = x - i * (E + 1);
+      const int i = div_small(x, inv_e1), e = x - i * (E + 1);
       if (e < E) {
         s.cnt[i * E + e] = v[u];
         a.cnt[i * E + e] = v[u];
