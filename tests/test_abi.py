@@ -164,3 +164,26 @@ def test_rank_entry_points_reject_bad_arguments_without_a_device(lib):
         zb.ERR_INVALID
     assert lib.zb_combine_rank(ctypes.byref(cfg), ctypes.byref(fake), tbl, 16, 8, None) == \
         zb.ERR_INVALID
+
+
+def test_plan_trace_conversion_on_the_host():
+    """zb.plan_trace turns the twelve stamps into microseconds from the first
+    kernel's start; a kernel that did not run (start left at all ones) is
+    None; a plan made without a trace is refused."""
+    import types
+
+    import torch
+    never = np.uint64(0xFFFFFFFFFFFFFFFF)
+    t = np.array([never, never, 0,              # k_zero: did not run
+                  1_000, 2_500, 3_000,          # k_hist
+                  1_800, 3_600, 14_000,         # k_planner
+                  4_000, 14_700, 17_500],       # k_assign
+                 dtype=np.uint64)
+    plan = types.SimpleNamespace(trace=torch.from_numpy(t.view(np.int64)))
+    tl = zb.plan_trace(plan)
+    assert tl["k_zero"] is None
+    assert tl["k_hist"] == {"start": 0.0, "released": 1.5, "end": 2.0}
+    assert tl["k_planner"] == {"start": 0.8, "released": 2.6, "end": 13.0}
+    assert tl["k_assign"] == {"start": 3.0, "released": 13.7, "end": 16.5}
+    with pytest.raises(zb.ZbError):
+        zb.plan_trace(types.SimpleNamespace(trace=None))
